@@ -1,0 +1,337 @@
+"""Benchmark of the QLoRA frozen-NF4 linear layer on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+One step = the whole hot path on one batch: NF4 + double quantisation of the
+bf16 weight, the forward (T = X·A, fused dequant GEMM Y = X·W_hatᵀ + sT·B) and
+the backward (U = dY·Bᵀ, fused dequant GEMM dX = dY·W_hat + sU·Aᵀ, dA, dB).
+Workload: a single 7B-class projection, W 4096 x 4096, X 4096 tokens
+(batch 4 x seq 1024), LoRA r = 64, alpha = 16, synthetic seeded inputs.
+value = algorithmic fwd+bwd flops per step / device time (TFLOP/s).
+
+Multi-GPU: the layer does not shard (one GPU per replica), so every rank runs
+its own replica of the workload and value sums the replicas' work over the
+slowest rank's time (weak scaling).  Rank 0 prints one JSON line.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = "QLoRA linear fwd+bwd TFLOP/s; packed-weight GB/s; fraction of roofline"
+WORKLOAD = "single 7B-class projection: W 4096x4096 NF4+DQ, X 4096 tokens (4x1024), LoRA r=64 alpha=16"
+
+
+def _peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+        return float(d["hbm_gbs"]), float(d["bf16_tflops"]), float(d.get("bf16_tflops_sustained", 0)), "measured"
+    except Exception:
+        return 6650.0, 1590.0, 1400.0, "fallback"
+
+
+class ClockSampler:
+    """nvidia-smi clocks / throttle reasons sampled while the timed region runs."""
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_id: str | None):
+        self.gpu_id = gpu_id
+        self.proc = None
+        self.path = None
+
+    def start(self):
+        try:
+            fd, self.path = tempfile.mkstemp(suffix=".csv")
+            os.close(fd)
+            cmd = ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits", "-lms", "50"]
+            if self.gpu_id:
+                cmd += ["-i", self.gpu_id]
+            self.proc = subprocess.Popen(cmd, stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+            time.sleep(0.3)
+        except Exception:
+            self.proc = None
+
+    def stop(self) -> dict:
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unavailable"]}
+        time.sleep(0.1)
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        rows = []
+        with open(self.path) as f:
+            for ln in f:
+                parts = [p.strip() for p in ln.split(",")]
+                if len(parts) >= 9:
+                    rows.append(parts)
+        os.unlink(self.path)
+        sm = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
+        mx = [float(r[2]) for r in rows if r[2].replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in rows for i in range(4) if r[5 + i].lower() == "active"})
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(mx) if mx else None,
+                "reasons": reasons, "samples": len(rows)}
+
+
+def _dist():
+    ws = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return ws, rank, local
+
+
+def run_ours(args):
+    import torch
+    import torch.distributed as dist
+    from datetime import timedelta
+
+    from bit_nf4_quantised_codebook_b200 import api, inputs
+
+    world, rank, local = _dist()
+    torch.cuda.set_device(local)
+    if world > 1:
+        dist.init_process_group("nccl", timeout=timedelta(seconds=120), device_id=torch.device("cuda", local))
+    api.lib()
+    dev = torch.device("cuda", local)
+    case = inputs.proj_7b()
+    M, N, K, r, s = case.M, case.N, case.K, case.r, case.s
+    flops = case.flops_fwd() + case.flops_bwd()
+
+    # Input sets rotated so that consecutive steps never find their inputs in L2
+    # (one set: W 33.5 MB + X 33.5 MB + dY 33.5 MB; outputs 67 MB more).
+    NSETS = 3
+    sets = []
+    for i in range(NSETS):
+        c = inputs.LinearCase(case.name, M, N, K, r, case.alpha, case.w_std, case.a_std, case.b_std,
+                              seed=case.seed + 10 * i)
+        sets.append({k: api.bits_to_tensor(getattr(c, k)(), dev) for k in ("W", "X", "A", "B", "dY")})
+    wq = api.alloc_weight(N, K, dev)
+    Y = torch.empty(M, N, dtype=torch.bfloat16, device=dev)
+    sT = torch.empty(M, r, dtype=torch.bfloat16, device=dev)
+    dX = torch.empty(M, K, dtype=torch.bfloat16, device=dev)
+    dA = torch.empty(K, r, dtype=torch.float32, device=dev)
+    dB = torch.empty(r, N, dtype=torch.float32, device=dev)
+    ws_q = torch.empty(api.qlora_workspace_size(api.QLORA_OP_QUANTIZE, 0, N, K, 0), dtype=torch.uint8, device=dev)
+    ws_f = torch.empty(api.qlora_workspace_size(api.QLORA_OP_FORWARD, M, N, K, r), dtype=torch.uint8, device=dev)
+    ws_b = torch.empty(api.qlora_workspace_size(api.QLORA_OP_BACKWARD, M, N, K, r), dtype=torch.uint8, device=dev)
+    err = api.new_error_word(dev)
+
+    def step(i, Win=None, Xin=None, Ain=None, Bin=None, dYin=None):
+        st = sets[i % NSETS]
+        Wt = st["W"] if Win is None else Win
+        Xt = st["X"] if Xin is None else Xin
+        At = st["A"] if Ain is None else Ain
+        Bt = st["B"] if Bin is None else Bin
+        dYt = st["dY"] if dYin is None else dYin
+        api.qlora_quantize(Wt, out=wq, ws=ws_q, dev_err=err)
+        api.qlora_linear_forward(wq, Xt, At, Bt, s, Y=Y, T_save=sT, ws=ws_f, dev_err=err)
+        api.qlora_linear_backward(wq, Xt, dYt, At, Bt, s, T_saved=sT, dX=dX, dA=dA, dB=dB, ws=ws_b, dev_err=err)
+
+    for i in range(args.warmup):
+        step(i)
+    torch.cuda.synchronize()
+    if int(err[0].item()) != 0:
+        raise RuntimeError(f"device error word {int(err[0].item())} during warm-up")
+
+    # dominant-kernel events (fused dequant GEMMs), one pair per step
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
+    gpu_id = None
+    try:
+        gpu_id = "GPU-" + str(torch.cuda.get_device_properties(local).uuid)
+    except Exception:
+        pass
+    sampler = ClockSampler(gpu_id)
+    sampler.start()
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    launches0 = api.qlora_kernel_launch_count()
+    t0 = torch.cuda.Event(enable_timing=True)
+    t1 = torch.cuda.Event(enable_timing=True)
+    t0.record()
+    for i in range(args.steps):
+        api.qlora_set_timing_events(*ev[i])
+        step(i)
+    t1.record()
+    torch.cuda.synchronize()
+    api.qlora_set_timing_events()
+    launches = api.qlora_kernel_launch_count() - launches0
+    if world > 1:
+        dist.barrier()
+    clocks = sampler.stop()
+    ms = t0.elapsed_time(t1)
+    fwd_ms = sum(e[0].elapsed_time(e[1]) for e in ev) / args.steps
+    bwd_ms = sum(e[2].elapsed_time(e[3]) for e in ev) / args.steps
+    if world > 1:
+        t = torch.tensor([ms], device=dev, dtype=torch.float64)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms = float(t.item())
+    torch.cuda.synchronize()
+    if int(err[0].item()) != 0:
+        raise RuntimeError(f"device error word {int(err[0].item())} during timing")
+    ms_step = ms / args.steps
+    value = flops * world / (ms_step * 1e-3) / 1e12
+
+    # end to end through the public API with pinned host buffers: H2D of the step's
+    # inputs (W, X, A, B, dY), the step, D2H of its results (Y, dX, dA, dB)
+    e2e_steps = max(3, min(20, args.steps // 10))
+    host_in = {k: torch.empty_like(v, device="cpu").pin_memory() for k, v in sets[0].items()}
+    for k in host_in:
+        host_in[k].copy_(sets[0][k])
+    dev_in = {k: torch.empty_like(v) for k, v in sets[0].items()}
+    host_out = [torch.empty_like(t, device="cpu").pin_memory() for t in (Y, dX, dA, dB)]
+    h2d = sum(t.numel() * t.element_size() for t in host_in.values())
+    d2h = sum(t.numel() * t.element_size() for t in host_out)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for i in range(e2e_steps):
+        for k in dev_in:
+            dev_in[k].copy_(host_in[k], non_blocking=True)
+        step(i, dev_in["W"], dev_in["X"], dev_in["A"], dev_in["B"], dev_in["dY"])
+        for h, d in zip(host_out, (Y, dX, dA, dB)):
+            h.copy_(d, non_blocking=True)
+    e1.record()
+    torch.cuda.synchronize()
+    e2e_ms = e0.elapsed_time(e1)
+    if world > 1:
+        t = torch.tensor([e2e_ms], device=dev, dtype=torch.float64)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        e2e_ms = float(t.item())
+    e2e_value = flops * world / (e2e_ms / e2e_steps * 1e-3) / 1e12
+
+    hbm, bf16_burst, bf16_sus, peak_src = _peaks()
+    # dominant kernel: the fused dequant GEMM of the backward (dX) or forward (Y), whichever is longer
+    dom = "bwd_dx" if bwd_ms >= fwd_ms else "fwd_y"
+    dom_ms = max(bwd_ms, fwd_ms)
+    dom_flops = 2.0 * M * N * K + 2.0 * M * r * (K if dom == "bwd_dx" else N)
+    achieved = dom_flops / (dom_ms * 1e-3) / 1e12
+    packed = wq.nbytes()
+
+    line = {
+        "metric": METRIC, "value": round(value, 3), "unit": "TFLOP/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_step, 4),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic (seeded numpy N(0,std) rounded to bf16)",
+        "config": {"workload": WORKLOAD, "M": M, "N": N, "K": K, "r": r, "alpha": case.alpha,
+                   "global_batch": 4 * world, "seq_len": 1024, "parallelism": f"replicas x{world} (no shard)",
+                   "step": "quantise(W) + forward + backward",
+                   "l2": f"inputs larger than L2: {NSETS} rotating input sets (W, X, dY 33.5 MB each) + 67 MB outputs"},
+        "packed_weight_gbs": round(2 * packed / (ms_step * 1e-3) / 1e9, 2),
+        "kernels": {"fwd_fused_ms": round(fwd_ms, 4), "bwd_fused_ms": round(bwd_ms, 4)},
+        "roofline": {"kernel": f"fused dequant GEMM ({dom})", "bound": "tensor",
+                     "achieved": round(achieved, 2), "peak": bf16_burst, "unit": "TFLOP/s",
+                     "frac": round(achieved / bf16_burst, 4), "peak_source": f"{peak_src} bf16 burst",
+                     "traffic": None},
+        "e2e": {"value": round(e2e_value, 3), "unit": "TFLOP/s", "h2d_bytes_per_step": h2d,
+                "d2h_bytes_per_step": d2h, "steps": e2e_steps},
+        "gpu_launches": int(launches),
+        "clocks": clocks,
+    }
+    if world == 1 and rank == 0 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline()
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+def _oracle_sample(rows: int, qrows: int | None = None):
+    """The oracle on a bounded sample of the workload: quantise + dequantise
+    `qrows` rows of the 4096 x 4096 weight (all of it by default), then forward +
+    backward for `rows` token rows through that (sub-)layer."""
+    from bit_nf4_quantised_codebook_b200 import inputs
+    from oracle import linear, nf4
+
+    case = inputs.proj_7b()
+    n = case.N if qrows is None else qrows
+    W, X, A, B, dY = case.W()[:n], case.X()[:rows], case.A(), case.B()[:, :n], case.dY()[:rows, :n]
+    t = time.perf_counter()
+    q = nf4.quantize_nf4(W)
+    what = nf4.dequantize_nf4(q)
+    linear.forward(X, what, A, B, case.s)
+    linear.backward(X, dY, what, A, B, case.s)
+    dt = time.perf_counter() - t
+    c = inputs.LinearCase(case.name, rows, n, case.K, case.r, case.alpha, case.w_std, case.a_std, case.b_std)
+    return dt, c.flops_fwd() + c.flops_bwd()
+
+
+def cpu_baseline(rows: int = 256) -> dict:
+    dt, fl = _oracle_sample(rows)
+    return {"value": round(fl / dt / 1e12, 6), "unit": "TFLOP/s", "cores": os.cpu_count(), "kind": "oracle",
+            "sample": f"quantise+dequantise the full 4096x4096 W, fwd+bwd on {rows} of 4096 token rows "
+                      f"(float64 numpy, BLAS threads = cores); {dt:.1f} s"}
+
+
+def run_reference(args):
+    """The oracle as the reference arm: every step is a bounded sample of the
+    workload (a slice of `n` weight rows and `n` token rows), sized so that the
+    whole --steps/--warmup run takes about two minutes of host time."""
+    world, rank, _ = _dist()
+    if rank != 0:
+        return
+    budget = 120.0 / max(1, args.steps + args.warmup)
+    n = 16
+    dt, _ = _oracle_sample(n, n)
+    while n < 1024 and dt * 2.2 < budget:
+        n *= 2
+        dt, _ = _oracle_sample(n, n)
+    for _ in range(args.warmup):
+        _oracle_sample(n, n)
+    tot_t, tot_f = 0.0, 0.0
+    for _ in range(args.steps):
+        dt, fl = _oracle_sample(n, n)
+        tot_t += dt
+        tot_f += fl
+    value = tot_f / tot_t / 1e12
+    line = {
+        "impl": "reference", "metric": METRIC, "value": round(value, 6), "unit": "TFLOP/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(tot_t / args.steps * 1e3, 3),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic (seeded numpy N(0,std) rounded to bf16)",
+        "config": {"workload": WORKLOAD, "M": 4096, "N": 4096, "K": 4096, "r": 64, "alpha": 16.0,
+                   "global_batch": 4, "seq_len": 1024, "parallelism": "cpu oracle"},
+        "cpu_baseline": {"value": round(value, 6), "unit": "TFLOP/s", "cores": os.cpu_count(), "kind": "oracle",
+                         "sample": f"per step: quantise+dequantise {n} weight rows (K=4096), fwd+bwd on {n} "
+                                   f"token rows through them"},
+        "e2e": {"value": round(value, 6), "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=1000)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_ours(args)
+
+
+if __name__ == "__main__":
+    main()

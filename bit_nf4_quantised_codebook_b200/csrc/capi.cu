@@ -1,0 +1,316 @@
+// capi.cu — the extern "C" boundary: argument validation, workspace layout,
+// tensor maps, and dispatch to the quantiser and the linear-layer launches.
+// Nothing here allocates device memory or synchronises the caller's stream.
+#include <algorithm>
+#include <atomic>
+#include <cstdint>
+#include <cstdlib>
+#include <cstring>
+#include <mutex>
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include "internal.h"
+#include "linear_plan.h"
+#include "nf4_decode.cuh"
+
+namespace qlora {
+namespace {
+
+struct Globals {
+  float levels[16];
+  float thresholds[15];
+  unsigned long long timeout_ns = 2000000000ull;  // 2 s per pipeline wait
+};
+
+Globals &globals() {
+  static Globals g;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    build_codebook_f32(g.levels, g.thresholds);
+    if (const char *env = std::getenv("QLORA_WAIT_TIMEOUT_MS")) {
+      const long long ms = std::atoll(env);
+      if (ms > 0) g.timeout_ns = static_cast<unsigned long long>(ms) * 1000000ull;
+    }
+  });
+  return g;
+}
+
+using EncodeTiledFn = CUresult (*)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *, const cuuint64_t *,
+                                   const cuuint64_t *, const cuuint32_t *, const cuuint32_t *, CUtensorMapInterleave,
+                                   CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void *p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  });
+  return fn;
+}
+
+bool encode_2d(CUtensorMap *m, CUtensorMapDataType dt, const void *ptr, uint64_t inner, uint64_t outer,
+               uint64_t row_bytes, uint32_t box_inner, uint32_t box_outer, CUtensorMapSwizzle sw) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return false;
+  const cuuint64_t dims[2] = {inner, outer};
+  const cuuint64_t strides[1] = {row_bytes};
+  const cuuint32_t box[2] = {box_inner, box_outer};
+  const cuuint32_t estr[2] = {1, 1};
+  return fn(m, dt, 2, const_cast<void *>(ptr), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, sw,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+int ceil_div(int64_t a, int64_t b) { return static_cast<int>((a + b - 1) / b); }
+
+SplitPlan choose(int64_t tiles, int64_t k_total, int target_ctas, int min_iters) {
+  SplitPlan sp;
+  sp.k_iters_total = static_cast<int>(k_total);
+  int64_t s = std::max<int64_t>(1, target_ctas / std::max<int64_t>(1, tiles));
+  s = std::min<int64_t>(s, std::max<int64_t>(1, k_total / std::max(1, min_iters)));
+  const int64_t kps = (k_total + s - 1) / s;
+  sp.k_iters = static_cast<int>(kps);
+  sp.splits = static_cast<int>((k_total + kps - 1) / kps);
+  return sp;
+}
+
+size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
+
+int device_sms() {
+  int dev = 0, sms = 148;
+  if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  return sms > 0 ? sms : 148;
+}
+
+bool device_ok() {
+  int dev = 0, major = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return false;
+  if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess) return false;
+  return major == 10;
+}
+
+bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+qlora_status check_weight(const qlora_nf4_weight *w) {
+  if (!w || !w->codes || !w->c2q || !w->c1 || !w->mean) return QLORA_ERR_INVALID_ARG;
+  if (w->N < 1 || w->K < 64) return QLORA_ERR_INVALID_ARG;
+  if (w->K % 64 != 0 || w->N > (1ll << 30) || w->K > (1ll << 30) || w->N * w->K > (1ll << 40))
+    return QLORA_ERR_UNSUPPORTED_SHAPE;
+  if (!aligned16(w->codes) || !aligned16(w->c2q) || !aligned16(w->c1) || !aligned16(w->mean))
+    return QLORA_ERR_MISALIGNED;
+  return QLORA_OK;
+}
+
+qlora_status check_linear(const qlora_nf4_weight *w, int64_t M, int r) {
+  qlora_status st = check_weight(w);
+  if (st != QLORA_OK) return st;
+  if (M < 1 || r < 1) return QLORA_ERR_INVALID_ARG;
+  if (r % 8 != 0 || r > 256 || w->N % 8 != 0 || M > (1ll << 30)) return QLORA_ERR_UNSUPPORTED_SHAPE;
+  return QLORA_OK;
+}
+
+std::atomic<uint64_t> g_launches{0};
+TimingHooks g_hooks;
+
+}  // namespace
+
+void count_launches(int n) { g_launches.fetch_add(static_cast<uint64_t>(n), std::memory_order_relaxed); }
+const TimingHooks &timing_hooks() { return g_hooks; }
+
+LinearPlan make_plan(int op, int64_t M, int64_t N, int64_t K, int r, int num_sms) {
+  LinearPlan pl;
+  size_t off = 0;
+  auto take = [&](size_t bytes) {
+    const size_t o = off;
+    off = align256(off + bytes);
+    return o;
+  };
+  if (op == QLORA_OP_QUANTIZE) {
+    const int64_t nb = N * K / 64;
+    const int64_t ng = (nb + 255) / 256;
+    int64_t size = 1;
+    while (size < ng) size *= 2;
+    pl.gsum_size = size;
+    pl.off_absmax = take(static_cast<size_t>(nb) * 4);
+    pl.off_gsum = take(static_cast<size_t>(size) * 8);
+    pl.bytes = off;
+    return pl;
+  }
+  pl.rpad = r <= 16 ? 16 : r <= 32 ? 32 : r <= 64 ? 64 : r <= 128 ? 128 : 256;
+  const int64_t mt = (M + 127) / 128;
+  pl.sp_t = choose(mt, K / 64, 2 * num_sms, 2);
+  pl.off_sT = take(static_cast<size_t>(M) * r * 2);
+  pl.off_t_part = take(static_cast<size_t>(pl.sp_t.splits) * M * pl.rpad * 4);
+  if (op == QLORA_OP_FORWARD) {
+    pl.sp_main = choose(mt * ((N + 255) / 256), K / 64, num_sms, 4);
+    if (pl.sp_main.splits > 1) pl.off_main_part = take(static_cast<size_t>(pl.sp_main.splits) * M * N * 4);
+  } else {
+    pl.sp_u = choose(mt, (N + 63) / 64, 2 * num_sms, 2);
+    pl.sp_dx = choose(mt * ((K + 255) / 256), (N + 63) / 64, num_sms, 4);
+    pl.sp_da = choose((K + 127) / 128, (M + 63) / 64, 2 * num_sms, 2);
+    pl.sp_db = choose((N + 127) / 128, (M + 63) / 64, 2 * num_sms, 2);
+    pl.off_sU = take(static_cast<size_t>(M) * r * 2);
+    pl.off_u_part = take(static_cast<size_t>(pl.sp_u.splits) * M * pl.rpad * 4);
+    if (pl.sp_dx.splits > 1) pl.off_main_part = take(static_cast<size_t>(pl.sp_dx.splits) * M * K * 4);
+    pl.off_da_part = take(static_cast<size_t>(pl.sp_da.splits) * K * pl.rpad * 4);
+    pl.off_db_part = take(static_cast<size_t>(pl.sp_db.splits) * N * pl.rpad * 4);
+  }
+  pl.bytes = off;
+  return pl;
+}
+
+bool map_bf16_kmajor(CUtensorMap *m, const void *ptr, int64_t inner, int64_t outer, int box_rows) {
+  return encode_2d(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, ptr, inner, outer, inner * 2, 64, box_rows,
+                   CU_TENSOR_MAP_SWIZZLE_128B);
+}
+bool map_bf16_mn(CUtensorMap *m, const void *ptr, int64_t inner, int64_t outer) {
+  return encode_2d(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, ptr, inner, outer, inner * 2, 64, 64,
+                   CU_TENSOR_MAP_SWIZZLE_128B);
+}
+bool map_codes(CUtensorMap *m, const void *codes, int64_t N, int64_t K, int box_bytes, int box_rows) {
+  return encode_2d(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, codes, K / 2, N, K / 2, box_bytes, box_rows,
+                   CU_TENSOR_MAP_SWIZZLE_NONE);
+}
+
+}  // namespace qlora
+
+using namespace qlora;
+
+extern "C" {
+
+const char *qlora_status_string(qlora_status st) {
+  switch (st) {
+    case QLORA_OK: return "ok";
+    case QLORA_ERR_INVALID_ARG: return "invalid argument";
+    case QLORA_ERR_UNSUPPORTED_SHAPE: return "unsupported shape";
+    case QLORA_ERR_MISALIGNED: return "pointer not 16-byte aligned";
+    case QLORA_ERR_CUDA: return "CUDA error";
+    case QLORA_ERR_WORKSPACE: return "workspace missing or too small";
+    case QLORA_ERR_NO_DEVICE: return "current device is not sm_100";
+  }
+  return "unknown status";
+}
+
+qlora_status qlora_build_codebook(float levels[16], float thresholds[15]) {
+  build_codebook_f32(levels, thresholds);
+  return QLORA_OK;
+}
+
+qlora_status qlora_nf4_sizes(int64_t N, int64_t K, size_t *codes_bytes, size_t *c2q_bytes, size_t *c1_bytes) {
+  if (N < 1 || K < 64) return QLORA_ERR_INVALID_ARG;
+  if (K % 64 != 0) return QLORA_ERR_UNSUPPORTED_SHAPE;
+  const int64_t nb = N * K / 64;
+  if (codes_bytes) *codes_bytes = static_cast<size_t>(N * K / 2);
+  if (c2q_bytes) *c2q_bytes = static_cast<size_t>(nb);
+  if (c1_bytes) *c1_bytes = static_cast<size_t>((nb + 255) / 256) * 4;
+  return QLORA_OK;
+}
+
+qlora_status qlora_workspace_size(int op, int64_t M, int64_t N, int64_t K, int r, size_t *bytes) {
+  if (!bytes || N < 1 || K < 64) return QLORA_ERR_INVALID_ARG;
+  if (K % 64 != 0) return QLORA_ERR_UNSUPPORTED_SHAPE;
+  if (op != QLORA_OP_QUANTIZE) {
+    if (M < 1 || r < 1) return QLORA_ERR_INVALID_ARG;
+    if (r % 8 != 0 || r > 256) return QLORA_ERR_UNSUPPORTED_SHAPE;
+  }
+  if (op < QLORA_OP_QUANTIZE || op > QLORA_OP_BACKWARD) return QLORA_ERR_INVALID_ARG;
+  *bytes = make_plan(op, M, N, K, r, device_sms()).bytes;
+  return QLORA_OK;
+}
+
+qlora_status qlora_quantize(const uint16_t *W, const qlora_nf4_weight *out, void *ws, size_t ws_bytes, int *dev_err,
+                            void *stream) {
+  if (!W) return QLORA_ERR_INVALID_ARG;
+  qlora_status st = check_weight(out);
+  if (st != QLORA_OK) return st;
+  if (!aligned16(W)) return QLORA_ERR_MISALIGNED;
+  if (!device_ok()) return QLORA_ERR_NO_DEVICE;
+  const LinearPlan pl = make_plan(QLORA_OP_QUANTIZE, 0, out->N, out->K, 0, device_sms());
+  if (!ws || ws_bytes < pl.bytes) return QLORA_ERR_WORKSPACE;
+  if (!aligned16(ws)) return QLORA_ERR_MISALIGNED;
+  Globals &g = globals();
+  Nf4Thresholds thr;
+  std::memcpy(thr.t, g.thresholds, sizeof(thr.t));
+  uint8_t *w8 = static_cast<uint8_t *>(ws);
+  const int64_t nb = out->N * out->K / 64;
+  cudaError_t e = launch_quantize(W, nb, out->codes, out->c2q, out->c1, out->mean,
+                                  reinterpret_cast<float *>(w8 + pl.off_absmax),
+                                  reinterpret_cast<double *>(w8 + pl.off_gsum), pl.gsum_size, thr, dev_err,
+                                  static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? QLORA_OK : QLORA_ERR_CUDA;
+}
+
+qlora_status qlora_dequantize(const qlora_nf4_weight *w, uint16_t *W_out, void *stream) {
+  qlora_status st = check_weight(w);
+  if (st != QLORA_OK) return st;
+  if (!W_out) return QLORA_ERR_INVALID_ARG;
+  if (!aligned16(W_out)) return QLORA_ERR_MISALIGNED;
+  if (!device_ok()) return QLORA_ERR_NO_DEVICE;
+  Globals &g = globals();
+  Nf4Levels lv;
+  std::memcpy(lv.q, g.levels, sizeof(lv.q));
+  cudaError_t e = launch_dequantize(w->codes, w->c2q, w->c1, w->mean, w->N * w->K / 64, lv, W_out,
+                                    static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? QLORA_OK : QLORA_ERR_CUDA;
+}
+
+static LaunchCtx make_ctx(int *dev_err, void *stream) {
+  Globals &g = globals();
+  LaunchCtx c;
+  c.stream = static_cast<cudaStream_t>(stream);
+  c.dev_err = dev_err;
+  c.timeout_ns = g.timeout_ns;
+  std::memcpy(c.levels.q, g.levels, sizeof(c.levels.q));
+  return c;
+}
+
+qlora_status qlora_linear_forward(const qlora_nf4_weight *w, const uint16_t *X, int64_t M, const uint16_t *A,
+                                  const uint16_t *B, int r, float s, uint16_t *Y, uint16_t *T_save, void *ws,
+                                  size_t ws_bytes, int *dev_err, void *stream) {
+  qlora_status st = check_linear(w, M, r);
+  if (st != QLORA_OK) return st;
+  if (!X || !A || !B || !Y) return QLORA_ERR_INVALID_ARG;
+  if (!aligned16(X) || !aligned16(A) || !aligned16(B) || !aligned16(Y) || (T_save && !aligned16(T_save)))
+    return QLORA_ERR_MISALIGNED;
+  if (!device_ok()) return QLORA_ERR_NO_DEVICE;
+  const LinearPlan pl = make_plan(QLORA_OP_FORWARD, M, w->N, w->K, r, device_sms());
+  if (!ws || ws_bytes < pl.bytes) return QLORA_ERR_WORKSPACE;
+  if (!aligned16(ws)) return QLORA_ERR_MISALIGNED;
+  cudaError_t e = run_forward(make_ctx(dev_err, stream), *w, X, M, A, B, r, s, Y, T_save, pl,
+                              static_cast<uint8_t *>(ws));
+  return e == cudaSuccess ? QLORA_OK : QLORA_ERR_CUDA;
+}
+
+qlora_status qlora_linear_backward(const qlora_nf4_weight *w, const uint16_t *X, const uint16_t *dY, int64_t M,
+                                   const uint16_t *A, const uint16_t *B, int r, float s, const uint16_t *T_saved,
+                                   uint16_t *dX, float *dA, float *dB, void *ws, size_t ws_bytes, int *dev_err,
+                                   void *stream) {
+  qlora_status st = check_linear(w, M, r);
+  if (st != QLORA_OK) return st;
+  if (!X || !dY || !A || !B || !dA || !dB) return QLORA_ERR_INVALID_ARG;
+  if (!aligned16(X) || !aligned16(dY) || !aligned16(A) || !aligned16(B) || !aligned16(dA) || !aligned16(dB) ||
+      (dX && !aligned16(dX)) || (T_saved && !aligned16(T_saved)))
+    return QLORA_ERR_MISALIGNED;
+  if (!device_ok()) return QLORA_ERR_NO_DEVICE;
+  const LinearPlan pl = make_plan(QLORA_OP_BACKWARD, M, w->N, w->K, r, device_sms());
+  if (!ws || ws_bytes < pl.bytes) return QLORA_ERR_WORKSPACE;
+  if (!aligned16(ws)) return QLORA_ERR_MISALIGNED;
+  cudaError_t e = run_backward(make_ctx(dev_err, stream), *w, X, dY, M, A, B, r, s, T_saved, dX, dA, dB, pl,
+                               static_cast<uint8_t *>(ws));
+  return e == cudaSuccess ? QLORA_OK : QLORA_ERR_CUDA;
+}
+
+uint64_t qlora_kernel_launch_count(void) { return g_launches.load(std::memory_order_relaxed); }
+
+qlora_status qlora_set_timing_events(void *fwd_begin, void *fwd_end, void *bwd_begin, void *bwd_end) {
+  g_hooks.fwd_begin = static_cast<cudaEvent_t>(fwd_begin);
+  g_hooks.fwd_end = static_cast<cudaEvent_t>(fwd_end);
+  g_hooks.bwd_begin = static_cast<cudaEvent_t>(bwd_begin);
+  g_hooks.bwd_end = static_cast<cudaEvent_t>(bwd_end);
+  return QLORA_OK;
+}
+
+}  // extern "C"

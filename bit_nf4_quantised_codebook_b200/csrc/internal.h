@@ -1,0 +1,33 @@
+// internal.h — declarations shared by the library's translation units.
+#pragma once
+#include <cstdint>
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include "../../include/qlora_nf4.h"
+
+namespace qlora {
+
+struct Nf4Levels;  // nf4_decode.cuh
+
+struct Nf4Thresholds {
+  float t[15];
+};
+
+// Process-wide diagnostics (capi.cu).
+void count_launches(int n);
+struct TimingHooks {
+  cudaEvent_t fwd_begin = nullptr, fwd_end = nullptr, bwd_begin = nullptr, bwd_end = nullptr;
+};
+const TimingHooks &timing_hooks();
+
+// Host code-book construction (codebook.cpp).
+void build_codebook_f64(double levels[16]);
+void build_codebook_f32(float levels[16], float thresholds[15]);
+
+cudaError_t launch_quantize(const uint16_t *W, int64_t nb, uint8_t *codes, uint8_t *c2q, float *c1, float *mean,
+                            float *ws_absmax, double *ws_gsum, int64_t gsum_size, const Nf4Thresholds &thr,
+                            int *dev_err, cudaStream_t st);
+cudaError_t launch_dequantize(const uint8_t *codes, const uint8_t *c2q, const float *c1, const float *mean,
+                              int64_t nb, const Nf4Levels &lv, uint16_t *out, cudaStream_t st);
+
+}  // namespace qlora

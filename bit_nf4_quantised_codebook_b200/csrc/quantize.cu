@@ -1,0 +1,169 @@
+// quantize.cu — blockwise NF4 quantiser with double quantisation, and the
+// standalone double-dequantiser.
+//
+// "QLoRA: Efficient Finetuning of Quantized LLMs" (intuitivepapers.ai):
+//   §Quantize in blocks  — flatten, cut into 64-element blocks, absmax per block;
+//   §NormalFloat         — each normalised weight goes to the nearest NF4 level;
+//   §Double quantization — block constants, mean-centred, become 8-bit floats in
+//                          groups of 256 with one float32 scale per group.
+//
+// Three launches, all HBM-streaming and deterministic:
+//   k_quant_blocks : one CTA per group of 256 blocks.  8 threads per block, one
+//                    16-byte load each; absmax by 3 xor-shuffles; codes by
+//                    threshold counting; nibble packing; per-group float64 sum of
+//                    the absmax values in block order (sequential, one thread).
+//   k_mean_tree    : one CTA, power-of-two pairwise tree over the group sums.
+//   k_double_quant : one CTA per group: centred constants, group absmax, S_g,
+//                    E4M3 codes (round to nearest even, saturating).
+#include <cstdint>
+#include <cuda_runtime.h>
+#include "internal.h"
+#include "nf4_decode.cuh"
+
+namespace qlora {
+
+__device__ __forceinline__ uint32_t e4m3_from_f32_satfinite(float x) {
+  uint16_t two;
+  asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(two) : "f"(x), "f"(x));
+  return two & 0xFFu;
+}
+
+__device__ __forceinline__ uint32_t nf4_code(float xh, const Nf4Thresholds &t) {
+  uint32_t c = 0;
+#pragma unroll
+  for (int i = 0; i < 15; ++i) c += (xh >= t.t[i]) ? 1u : 0u;
+  return c;
+}
+
+__global__ void __launch_bounds__(256) k_quant_blocks(const uint16_t *__restrict__ W, int64_t nb,
+                                                       uint8_t *__restrict__ codes, float *__restrict__ absmax,
+                                                       double *__restrict__ gsum, Nf4Thresholds thr,
+                                                       int *dev_err) {
+  __shared__ float s_amax[256];
+  const int64_t g = blockIdx.x;
+  const int part = threadIdx.x & 7;  // 8-element chunk of the block
+  const int sub = threadIdx.x >> 3;  // block within the pass
+  bool bad = false;
+#pragma unroll 1
+  for (int pass = 0; pass < 8; ++pass) {
+    const int lb = pass * 32 + sub;
+    const int64_t b = g * 256 + lb;
+    const bool valid = b < nb;
+    uint4 raw = make_uint4(0, 0, 0, 0);
+    if (valid) raw = __ldg(reinterpret_cast<const uint4 *>(W + b * 64) + part);
+    const uint32_t u[4] = {raw.x, raw.y, raw.z, raw.w};
+    float x[8];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      x[2 * i] = __uint_as_float(u[i] << 16);
+      x[2 * i + 1] = __uint_as_float(u[i] & 0xFFFF0000u);
+    }
+    float amax = 0.f;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      const float a = fabsf(x[i]);
+      bad |= !(a <= 3.402823466e38f);
+      amax = fmaxf(amax, a);
+    }
+    amax = fmaxf(amax, __shfl_xor_sync(0xFFFFFFFFu, amax, 1));
+    amax = fmaxf(amax, __shfl_xor_sync(0xFFFFFFFFu, amax, 2));
+    amax = fmaxf(amax, __shfl_xor_sync(0xFFFFFFFFu, amax, 4));
+    uint32_t packed = 0;
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const float xa = amax == 0.f ? 0.f : __fdiv_rn(x[2 * i], amax);
+      const float xb = amax == 0.f ? 0.f : __fdiv_rn(x[2 * i + 1], amax);
+      const uint32_t byte = (nf4_code(xa, thr) << 4) | nf4_code(xb, thr);
+      packed |= byte << (8 * i);
+    }
+    if (valid) {
+      reinterpret_cast<uint32_t *>(codes + b * 32)[part] = packed;
+      if (part == 0) absmax[b] = amax;
+    }
+    if (part == 0) s_amax[lb] = valid ? amax : 0.f;
+  }
+  if (bad && dev_err) atomicOr(dev_err, QLORA_DEVERR_NONFINITE);
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    const int64_t cnt = nb - g * 256 < 256 ? nb - g * 256 : 256;
+    double acc = 0.0;
+    for (int j = 0; j < cnt; ++j) acc = __dadd_rn(acc, static_cast<double>(s_amax[j]));
+    gsum[g] = acc;
+  }
+}
+
+__global__ void __launch_bounds__(1024) k_mean_tree(double *__restrict__ a, int64_t ng, int64_t size, int64_t nb,
+                                                     float *__restrict__ mean) {
+  for (int64_t i = ng + threadIdx.x; i < size; i += blockDim.x) a[i] = 0.0;
+  __syncthreads();
+  for (int64_t h = size / 2; h >= 1; h /= 2) {
+    for (int64_t i = threadIdx.x; i < h; i += blockDim.x) a[i] = __dadd_rn(a[i], a[i + h]);
+    __syncthreads();
+  }
+  if (threadIdx.x == 0) *mean = __double2float_rn(__ddiv_rn(a[0], static_cast<double>(nb)));
+}
+
+__global__ void __launch_bounds__(256) k_double_quant(const float *__restrict__ absmax, int64_t nb,
+                                                       const float *__restrict__ mean, uint8_t *__restrict__ c2q,
+                                                       float *__restrict__ c1) {
+  __shared__ float s_red[8];
+  const int64_t g = blockIdx.x;
+  const int64_t b = g * 256 + threadIdx.x;
+  const bool valid = b < nb;
+  const float mu = *mean;
+  const float dev = valid ? __fsub_rn(absmax[b], mu) : 0.f;
+  float a = fabsf(dev);
+#pragma unroll
+  for (int o = 16; o >= 1; o >>= 1) a = fmaxf(a, __shfl_xor_sync(0xFFFFFFFFu, a, o));
+  if ((threadIdx.x & 31) == 0) s_red[threadIdx.x >> 5] = a;
+  __syncthreads();
+  float amax = s_red[0];
+#pragma unroll
+  for (int i = 1; i < 8; ++i) amax = fmaxf(amax, s_red[i]);
+  const float sg = __fdiv_rn(amax, 448.0f);
+  uint32_t e = 0;
+  if (sg != 0.f) e = e4m3_from_f32_satfinite(__fdiv_rn(dev, sg));
+  if (valid) c2q[b] = static_cast<uint8_t>(e);
+  if (threadIdx.x == 0) c1[g] = sg;
+}
+
+__global__ void __launch_bounds__(256) k_dequant(const uint8_t *__restrict__ codes, const uint8_t *__restrict__ c2q,
+                                                  const float *__restrict__ c1, const float *__restrict__ mean,
+                                                  int64_t nb, Nf4Levels lv, uint16_t *__restrict__ out) {
+  const int64_t b = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+  if (b >= nb) return;
+  const float c2h = reconstruct_c2(c2q[b], c1[b >> 8], *mean);
+  const BlockLut lut = make_lut(c2h, lv);
+  const uint4 *cp = reinterpret_cast<const uint4 *>(codes + b * 32);
+  const uint4 q0 = __ldg(cp), q1 = __ldg(cp + 1);
+  const uint32_t w[8] = {q0.x, q0.y, q0.z, q0.w, q1.x, q1.y, q1.z, q1.w};
+  uint4 *op = reinterpret_cast<uint4 *>(out + b * 64);
+#pragma unroll
+  for (int c = 0; c < 8; ++c) {
+    uint32_t o[4];
+    decode8(w[c], lut, o);
+    op[c] = make_uint4(o[0], o[1], o[2], o[3]);
+  }
+}
+
+// ---------------------------------------------------------------- host launchers
+cudaError_t launch_quantize(const uint16_t *W, int64_t nb, uint8_t *codes, uint8_t *c2q, float *c1, float *mean,
+                            float *ws_absmax, double *ws_gsum, int64_t gsum_size, const Nf4Thresholds &thr,
+                            int *dev_err, cudaStream_t st) {
+  const int64_t ng = (nb + 255) / 256;
+  k_quant_blocks<<<static_cast<unsigned>(ng), 256, 0, st>>>(W, nb, codes, ws_absmax, ws_gsum, thr, dev_err);
+  k_mean_tree<<<1, 1024, 0, st>>>(ws_gsum, ng, gsum_size, nb, mean);
+  k_double_quant<<<static_cast<unsigned>(ng), 256, 0, st>>>(ws_absmax, nb, mean, c2q, c1);
+  count_launches(3);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_dequantize(const uint8_t *codes, const uint8_t *c2q, const float *c1, const float *mean,
+                              int64_t nb, const Nf4Levels &lv, uint16_t *out, cudaStream_t st) {
+  const int64_t grid = (nb + 255) / 256;
+  k_dequant<<<static_cast<unsigned>(grid), 256, 0, st>>>(codes, c2q, c1, mean, nb, lv, out);
+  count_launches(1);
+  return cudaGetLastError();
+}
+
+}  // namespace qlora

@@ -1,0 +1,185 @@
+/*
+ * qlora_nf4.h — C ABI of the B200 (sm_100a) QLoRA frozen-NF4 linear layer.
+ *
+ * The method (web pages on QLoRA; main source "QLoRA: Efficient Finetuning of
+ * Quantized LLMs", intuitivepapers.ai):
+ *   - §NormalFloat: a 16-level NormalFloat-4 code book (7 negative levels, an
+ *     exact zero, 8 positive levels, ends at -1 and +1);
+ *   - §Quantize in blocks: the flattened weight is cut into blocks of 64
+ *     consecutive elements, each with its own absmax constant;
+ *   - §Double quantization: the block constants, mean-centred, are stored as
+ *     8-bit floats in groups of 256 with one float32 scale per group;
+ *   - §The QLoRA layer, end to end: Y = X·W + s·(X·L1)·L2 with W dequantised
+ *     to bfloat16 on the fly; backward gives dX through W and the adapter,
+ *     and gradients for L1, L2 only.
+ *
+ * Conventions of this library:
+ *   W  [N, K]  frozen weight, bfloat16, row-major (out x in, as a framework
+ *              Linear stores it); quantisation blocks run along the flat
+ *              row-major index, so K must be a multiple of 64.
+ *   X  [M, K]  activations, bfloat16 row-major.  M >= 1 tokens.
+ *   A  [K, r]  first adapter factor (the pages' L1), bfloat16 row-major.
+ *   B  [r, N]  second adapter factor (L2), bfloat16 row-major.
+ *   s          adapter scale alpha / r.
+ *   Y  [M, N] = X·W_hatᵀ + s·(X·A)·B, bfloat16 (float32 accumulation).
+ *   W_hat = doubleDequant(W_NF4), bfloat16, never written to HBM by the
+ *   forward or backward pass.
+ *
+ * Stored NF4 weight (all buffers on the device, owned by the caller):
+ *   codes  N·K/2 bytes: element 2j of the flat weight in the HIGH nibble of
+ *          byte j, element 2j+1 in the LOW nibble; 16-byte aligned.
+ *   c2q    N·K/64 bytes: OCP FP8 E4M3FN code e_b of each block's centred
+ *          absmax (block b = flat elements [64b, 64b+64)).
+ *   c1     ceil(N·K/64/256) float32: group scale S_g (group g = blocks
+ *          [256g, 256g+256) of the flat block index; may straddle rows; the
+ *          last group may be partial).
+ *   mean   1 float32: mu, the mean of all block absmax values.
+ *   Reconstruction: c2_hat_b = fmaf(e_b, S_g, mu);
+ *                   w_hat = bf16_rn(float32(level[code] · c2_hat_b)).
+ *
+ * bfloat16 tensors are passed as uint16_t bit patterns.  All sizes are in
+ * elements unless stated.  Every device pointer must be 16-byte aligned.
+ * `stream` is a cudaStream_t (NULL = legacy default stream).  Every call is
+ * asynchronous on `stream`, never synchronises and never allocates.
+ *
+ * Errors: the return value reports host-side validation and launch errors;
+ * nothing is launched when validation fails.  Conditions detected on the
+ * device are OR-ed into *dev_err (a device int, nullable) as QLORA_DEVERR_*
+ * bits; read it after synchronising the stream.
+ */
+#ifndef QLORA_NF4_H
+#define QLORA_NF4_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  QLORA_OK = 0,
+  QLORA_ERR_INVALID_ARG = 1,       /* null pointer, non-positive size, bad op */
+  QLORA_ERR_UNSUPPORTED_SHAPE = 2, /* K % 64 != 0, r not in {8,16,...,256}, N % 8 != 0, overflow */
+  QLORA_ERR_MISALIGNED = 3,        /* a device pointer is not 16-byte aligned */
+  QLORA_ERR_CUDA = 4,              /* a CUDA runtime / driver call failed */
+  QLORA_ERR_WORKSPACE = 5,         /* workspace missing or smaller than qlora_workspace_size() */
+  QLORA_ERR_NO_DEVICE = 6          /* the current device is not sm_100 */
+} qlora_status;
+
+/* Bits OR-ed into *dev_err by kernels. */
+#define QLORA_DEVERR_NONFINITE 1   /* the weight given to qlora_quantize held Inf/NaN */
+#define QLORA_DEVERR_TIMEOUT   2   /* a pipeline wait exceeded its bound; outputs are undefined */
+
+typedef struct qlora_nf4_weight {
+  int64_t N, K;      /* logical shape of W */
+  uint8_t *codes;    /* N*K/2 bytes   */
+  uint8_t *c2q;      /* N*K/64 bytes  */
+  float *c1;         /* ceil(N*K/16384) floats */
+  float *mean;       /* 1 float       */
+} qlora_nf4_weight;
+
+enum { QLORA_OP_QUANTIZE = 0, QLORA_OP_FORWARD = 1, QLORA_OP_BACKWARD = 2 };
+
+/* Human-readable name of a status code (static string). */
+const char *qlora_status_string(qlora_status st);
+
+/*
+ * qlora_build_codebook — host only.  §NormalFloat (intuitivepapers.ai): the
+ * offset recipe (tail probability 0.9677083; 8 positive normal quantiles at
+ * probabilities evenly spaced from the offset towards 1/2, 7 negative ones
+ * likewise, an exact 0; sorted; divided by the largest magnitude).  Quantiles
+ * come from Wichura's AS 241 (1988) refined by one Newton step on erfc, in
+ * float64, then rounded to float32.
+ * levels[16]    : ascending, levels[0] = -1, levels[7] = 0, levels[15] = +1.
+ * thresholds[15]: thresholds[i] = smallest float32 strictly above the exact
+ *                 midpoint (levels[i]+levels[i+1])/2, so that
+ *                 code(x) = #{i : x >= thresholds[i]} is the nearest level with
+ *                 ties going to the lower index.
+ * Either pointer may be NULL.  Returns QLORA_OK.
+ */
+qlora_status qlora_build_codebook(float levels[16], float thresholds[15]);
+
+/* Byte sizes of the three stored arrays of an N x K weight (mean is 4 bytes). */
+qlora_status qlora_nf4_sizes(int64_t N, int64_t K, size_t *codes_bytes, size_t *c2q_bytes,
+                             size_t *c1_bytes);
+
+/*
+ * Workspace bytes an operation needs (op = QLORA_OP_*; M and r are ignored for
+ * QLORA_OP_QUANTIZE).  The caller allocates it (16-byte aligned) and passes it
+ * to the call; it holds no state between calls.
+ */
+qlora_status qlora_workspace_size(int op, int64_t M, int64_t N, int64_t K, int r, size_t *bytes);
+
+/*
+ * qlora_quantize — §Quantize in blocks, §NormalFloat, §Double quantization.
+ * W: device, N*K bfloat16 (the shape comes from out->N, out->K).
+ * Per block: c2 = max|w| (float32); x = float32(w / c2); code = nearest level
+ * (ties to the lower index; an all-zero block gives the zero level, 7).
+ * Second level: mu = mean of all c2 in a fixed order (per group of 256 blocks
+ * a sequential float64 sum, then a power-of-two pairwise tree; float64 divide
+ * by the block count, rounded to float32); dev = float32(c2 - mu);
+ * S_g = float32(max|dev| over the group / 448); e = E4M3(dev / S_g) with
+ * round-to-nearest-even and saturation (S_g = 0 gives e = 0).
+ * Writes out->codes, out->c2q, out->c1, out->mean.  A non-finite weight sets
+ * QLORA_DEVERR_NONFINITE in *dev_err (outputs then unspecified).
+ * Deterministic: identical inputs give identical bits.
+ */
+qlora_status qlora_quantize(const uint16_t *W, const qlora_nf4_weight *out, void *ws,
+                            size_t ws_bytes, int *dev_err, void *stream);
+
+/*
+ * qlora_dequantize — doubleDequant of §The QLoRA layer, end to end, written
+ * out to HBM (for tests and inspection; the layer itself never does this).
+ * W_out: device, N*K bfloat16.
+ */
+qlora_status qlora_dequantize(const qlora_nf4_weight *w, uint16_t *W_out, void *stream);
+
+/*
+ * qlora_linear_forward — §LoRA and §The QLoRA layer, end to end (forward).
+ *   T_save (nullable, device, M x r bfloat16) receives bf16(s · X·A), the
+ *   scaled adapter activation the backward pass reuses.
+ *   Y (device, M x N bfloat16) = X·W_hatᵀ + (bf16(s·X·A))·B, float32 accumulate.
+ * W_hat is produced tile by tile inside the GEMM (tensor cores, tcgen05) and
+ * never stored.  ws: qlora_workspace_size(QLORA_OP_FORWARD, ...) bytes.
+ */
+qlora_status qlora_linear_forward(const qlora_nf4_weight *w, const uint16_t *X, int64_t M,
+                                  const uint16_t *A, const uint16_t *B, int r, float s,
+                                  uint16_t *Y, uint16_t *T_save, void *ws, size_t ws_bytes,
+                                  int *dev_err, void *stream);
+
+/*
+ * qlora_linear_backward — §The QLoRA layer, end to end (backward listing).
+ *   U  = dY·Bᵀ                                   (M x r)
+ *   dX = dY·W_hat + bf16(s·U)·Aᵀ                 (M x K bfloat16; nullable = skip)
+ *   dA = Xᵀ·bf16(s·U)                            (K x r float32)
+ *   dB = T_savedᵀ·dY                             (r x N float32)
+ * T_saved is the forward's T_save = bf16(s·X·A); NULL recomputes it from X and A.
+ * No gradient for W is formed.  ws: qlora_workspace_size(QLORA_OP_BACKWARD, ...).
+ */
+qlora_status qlora_linear_backward(const qlora_nf4_weight *w, const uint16_t *X,
+                                   const uint16_t *dY, int64_t M, const uint16_t *A,
+                                   const uint16_t *B, int r, float s, const uint16_t *T_saved,
+                                   uint16_t *dX, float *dA, float *dB, void *ws, size_t ws_bytes,
+                                   int *dev_err, void *stream);
+
+/* ---------------------------------------------------------------- diagnostics
+ * (no counterpart on the pages: instrumentation for measurement)            */
+
+/* Number of kernels this library has launched in this process so far. */
+uint64_t qlora_kernel_launch_count(void);
+
+/*
+ * Optional timing hooks.  Each argument is a cudaEvent_t or NULL.  While set,
+ * every qlora_linear_forward records fwd_begin / fwd_end on its stream
+ * immediately before / after launching the fused dequant GEMM (Y), and every
+ * qlora_linear_backward records bwd_begin / bwd_end around the fused dequant
+ * GEMM that produces dX.  Passing all NULL disables the hooks.  The setting is
+ * process-wide and not thread-safe.
+ */
+qlora_status qlora_set_timing_events(void *fwd_begin, void *fwd_end, void *bwd_begin, void *bwd_end);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* QLORA_NF4_H */

@@ -1,0 +1,90 @@
+"""Host-side checks of the C ABI: the library loads, exports every symbol the
+header declares, builds the same code book as the oracle, and rejects bad
+arguments before launching anything (no GPU needed)."""
+import ctypes
+import os
+import re
+import subprocess
+
+import numpy as np
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "qlora_nf4.h")
+
+
+@pytest.fixture(scope="module")
+def api():
+    from bit_nf4_quantised_codebook_b200 import build
+    build.build()
+    from bit_nf4_quantised_codebook_b200 import api as a
+    return a
+
+
+def _declared():
+    src = open(HEADER).read()
+    return sorted(set(re.findall(r"^(?:qlora_status|const char \*)\s*(qlora_\w+)\s*\(", src, re.M)))
+
+
+def test_header_declares_expected_entry_points():
+    names = _declared()
+    for n in ["qlora_build_codebook", "qlora_quantize", "qlora_dequantize", "qlora_linear_forward",
+              "qlora_linear_backward", "qlora_nf4_sizes", "qlora_workspace_size", "qlora_status_string"]:
+        assert n in names
+
+
+def test_library_exports_every_declared_symbol(api):
+    L = api.lib()
+    out = subprocess.run(["nm", "-D", "--defined-only", api.LIB_PATH], capture_output=True, text=True).stdout
+    exported = set(ln.split()[-1] for ln in out.splitlines() if ln.strip())
+    for n in _declared():
+        assert n in exported, n
+        assert hasattr(L, n)
+
+
+def test_codebook_matches_oracle(api):
+    from oracle import nf4
+    lv, th = api.qlora_build_codebook()
+    lv = np.array(lv, np.float32)
+    th = np.array(th, np.float32)
+    assert np.array_equal(lv.view(np.uint32), nf4.nf4_levels().view(np.uint32))
+    assert np.array_equal(th.view(np.uint32), nf4.nf4_thresholds(nf4.nf4_levels()).view(np.uint32))
+
+
+def test_sizes(api):
+    from oracle import nf4
+    cb, qb, sb = api.qlora_nf4_sizes(4096, 4096)
+    assert cb + qb + sb + 4 == nf4.storage_bytes(4096, 4096)
+    cb, qb, sb = api.qlora_nf4_sizes(3, 6400)
+    assert (cb, qb, sb) == (9600, 300, 8)
+
+
+def test_validation_errors(api):
+    L = api.lib()
+    n = ctypes.c_size_t()
+    assert L.qlora_nf4_sizes(16, 100, None, None, None) == 2          # K % 64
+    assert L.qlora_workspace_size(1, 4, 16, 64, 12, ctypes.byref(n)) == 2   # r % 8
+    assert L.qlora_workspace_size(1, 4, 16, 64, 8, None) == 1
+    assert L.qlora_workspace_size(7, 4, 16, 64, 8, ctypes.byref(n)) == 1
+    assert L.qlora_workspace_size(1, 4096, 4096, 4096, 64, ctypes.byref(n)) == 0 and n.value > 0
+    w = api._Weight(16, 100, 16, 16, 16, 16)
+    assert L.qlora_quantize(16, ctypes.byref(w), 16, 1 << 20, None, None) == 2
+    w = api._Weight(16, 128, 16, 16, 16, 16)
+    assert L.qlora_quantize(None, ctypes.byref(w), 16, 1 << 20, None, None) == 1
+    w = api._Weight(16, 128, 0, 16, 16, 16)
+    assert L.qlora_quantize(16, ctypes.byref(w), 16, 1 << 20, None, None) == 1
+    w = api._Weight(16, 128, 17, 16, 16, 16)
+    assert L.qlora_quantize(16, ctypes.byref(w), 16, 1 << 20, None, None) == 3
+    w = api._Weight(12, 128, 16, 16, 16, 16)                           # N % 8 for the linear layer
+    assert L.qlora_linear_forward(ctypes.byref(w), 16, 4, 16, 16, 8, ctypes.c_float(1.0), 16, None, 16,
+                                  1 << 20, None, None) == 2
+    assert api.lib().qlora_status_string(3) == b"pointer not 16-byte aligned"
+
+
+def test_product_path_has_no_cpu_fallback():
+    """The binding never imports the oracle; the package refuses to run without the library."""
+    pkg = os.path.join(ROOT, "bit_nf4_quantised_codebook_b200")
+    for f in os.listdir(pkg):
+        if f.endswith(".py"):
+            txt = open(os.path.join(pkg, f)).read()
+            assert "import oracle" not in txt and "from oracle" not in txt, f
