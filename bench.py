@@ -151,6 +151,9 @@ def run_ours(args):
 
     # dominant-kernel events (fused dequant GEMMs), one pair per step
     ev = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
+    for quad in ev:          # torch creates events lazily: record once so each has a handle
+        for e in quad:
+            e.record()
     gpu_id = None
     try:
         gpu_id = "GPU-" + str(torch.cuda.get_device_properties(local).uuid)
