@@ -145,11 +145,13 @@ LinearPlan make_plan(int op, int64_t M, int64_t N, int64_t K, int r, int num_sms
   pl.off_sT = take(static_cast<size_t>(M) * r * 2);
   pl.off_t_part = take(static_cast<size_t>(pl.sp_t.splits) * M * pl.rpad * 4);
   if (op == QLORA_OP_FORWARD) {
-    pl.sp_main = choose(mt * ((N + 255) / 256), K / 64, num_sms, 4);
+    pl.pair_main = M > 128;
+    pl.sp_main = choose((pl.pair_main ? 2 * ((M + 255) / 256) : mt) * ((N + 255) / 256), K / 64, num_sms, 4);
     if (pl.sp_main.splits > 1) pl.off_main_part = take(static_cast<size_t>(pl.sp_main.splits) * M * N * 4);
   } else {
     pl.sp_u = choose(mt, (N + 63) / 64, 2 * num_sms, 2);
-    pl.sp_dx = choose(mt * ((K + 255) / 256), (N + 63) / 64, num_sms, 4);
+    pl.pair_dx = M > 128;
+    pl.sp_dx = choose((pl.pair_dx ? 2 * ((M + 255) / 256) : mt) * ((K + 255) / 256), (N + 63) / 64, num_sms, 4);
     pl.sp_da = choose((K + 127) / 128, (M + 63) / 64, 2 * num_sms, 2);
     pl.sp_db = choose((N + 127) / 128, (M + 63) / 64, 2 * num_sms, 2);
     pl.off_sU = take(static_cast<size_t>(M) * r * 2);
@@ -170,9 +172,9 @@ bool map_bf16_mn(CUtensorMap *m, const void *ptr, int64_t inner, int64_t outer) 
   return encode_2d(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, ptr, inner, outer, inner * 2, 64, 64,
                    CU_TENSOR_MAP_SWIZZLE_128B);
 }
-bool map_codes(CUtensorMap *m, const void *codes, int64_t N, int64_t K, int box_bytes, int box_rows) {
+bool map_codes(CUtensorMap *m, const void *codes, int64_t N, int64_t K, int box_bytes, int box_rows, bool swizzle64) {
   return encode_2d(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, codes, K / 2, N, K / 2, box_bytes, box_rows,
-                   CU_TENSOR_MAP_SWIZZLE_NONE);
+                   swizzle64 ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_NONE);
 }
 
 }  // namespace qlora

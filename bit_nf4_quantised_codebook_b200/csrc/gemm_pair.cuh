@@ -1,0 +1,296 @@
+// gemm_pair.cuh — the fused dequant GEMM on a CTA pair (cluster of 2, tcgen05
+// cta_group::2): one 256 x 256 output tile per pair.
+//
+//   D[256 tokens x 256] = sum_k Aop[256 x k] · W_hat-side[256 x k]ᵀ  (+ LoRA tail)
+//
+// Each CTA of the pair stages its own 128 token rows of the activation (TMA)
+// and dequantises its own 128 rows of the W-side operand; the leader CTA issues
+// the pair MMA, which reads both CTAs' shared memory at the same offsets and
+// writes each CTA's 128 x 256 accumulator slice into that CTA's TMEM.  Against
+// a one-CTA 128 x 256 tile this halves the dequantisation work per flop and the
+// W-side operand bytes each SM stages.
+//
+// Roles per CTA (320 threads):
+//   warp 0      TMA producer (own activation half + own packed-code half, or
+//               the LoRA operand halves) into a STAGES-deep ring; local
+//               full[] barriers.
+//   warp 1      TMEM allocation (pair); in the leader, the MMA issuer: waits
+//               ready[s] (8 warp arrivals: 4 per CTA), issues 4 pair MMAs,
+//               commits empty[s] to both CTAs (multicast).
+//   warps 2..9  two dequant groups of 4 warps taking alternate stages: wait the
+//               local full[s], expand 128 rows x 64 codes to bf16 in the
+//               swizzled UMMA layout, fence to the async proxy, arrive on the
+//               leader's ready[s].  Warps 2..5 then run the epilogue.
+// Shared-memory bank use: K-major code rows are read in an order that gives
+// the 8 threads of each 128-bit phase distinct banks; MN-major code tiles are
+// staged with the TMA 64-byte swizzle for the same reason.
+#pragma once
+#include <cstdint>
+#include <cuda.h>
+#include "gemm.cuh"
+
+namespace qlora {
+
+template <int STAGES_, int BMODE_, int LORA_, int OUT_>
+struct PairCfg {
+  static constexpr int STAGES = STAGES_;
+  static constexpr int BMODE = BMODE_;
+  static constexpr int LORA = LORA_;
+  static constexpr int OUT = OUT_;
+  static constexpr int BN = 256;  // pair N
+  static constexpr bool B_MN = BMODE == B_DQ_MN;
+  static constexpr int A_BYTES = 128 * 64 * 2;
+  static constexpr int B_BYTES = 128 * 64 * 2;
+  static constexpr int C_BYTES = 4096;
+  static constexpr int STAGE_BYTES = A_BYTES + B_BYTES + C_BYTES;
+  static constexpr int NUM_THREADS = 320;
+  static constexpr int TMEM_COLS = 256;
+  static constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + 256 + 1024;
+  static_assert(BMODE == B_DQ_K || BMODE == B_DQ_MN, "pair kernel dequantises its W-side operand");
+  static_assert(STAGE_BYTES % 1024 == 0, "swizzle atoms need 1 KiB alignment");
+};
+
+template <class C>
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(C::NUM_THREADS, 1)
+    gemm_pair_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constant__ CUtensorMap map_codes,
+                     const __grid_constant__ CUtensorMap map_a2, const __grid_constant__ CUtensorMap map_b2,
+                     const GemmParams p) {
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint64_t *bars = reinterpret_cast<uint64_t *>(smem + C::STAGES * C::STAGE_BYTES);
+  uint64_t *full = bars;                      // local TMA landed
+  uint64_t *empty = bars + C::STAGES;         // pair MMAs finished with the stage (multicast commit)
+  uint64_t *ready = bars + 2 * C::STAGES;     // leader only: both CTAs' operands staged
+  uint64_t *acc_full = bars + 3 * C::STAGES;  // all pair MMAs of the tile done (multicast commit)
+  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 3 * C::STAGES + 1);
+  volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const uint32_t rank = cluster_ctarank();
+  const bool leader = rank == 0;
+  const int m0 = blockIdx.x * 128;            // this CTA's token rows
+  const int n0 = blockIdx.y * C::BN;          // the pair's W-side tile
+  const int nh0 = n0 + 128 * static_cast<int>(rank);  // this CTA's half of it
+  const int split = blockIdx.z;
+  const int kb_begin = split * p.k_iters;
+  int n_main = p.k_iters_total - kb_begin;
+  if (n_main > p.k_iters) n_main = p.k_iters;
+  const int n_lora = (C::LORA != LORA_NONE && split == 0) ? (p.lora_r + 63) / 64 : 0;
+  const int n_total = n_main + n_lora;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < C::STAGES; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+      mbar_init(&ready[s], 8);
+    }
+    mbar_init(acc_full, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 0 && lane == 0) {
+    tma_prefetch_desc(&map_a);
+    tma_prefetch_desc(&map_codes);
+    if (C::LORA != LORA_NONE) {
+      tma_prefetch_desc(&map_a2);
+      tma_prefetch_desc(&map_b2);
+    }
+  }
+  if (warp == 1) {
+    tmem_alloc_pair(tmem_slot, C::TMEM_COLS);
+    tmem_relinquish_pair();
+  }
+  tc_fence_before();
+  __syncthreads();
+  cluster_sync();
+  tc_fence_after();
+  const uint32_t tmem_acc = *tmem_slot;
+  const uint32_t smem_base = smem_u32(smem);
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ TMA producer
+    if (lane == 0) {
+      int issued = 0;
+      for (int it = 0; it < n_total; ++it) {
+        const int s = it % C::STAGES;
+        const uint32_t ph = (it / C::STAGES) & 1;
+        if (!mbar_wait_cluster_bounded(&empty[s], ph ^ 1, abort_flag, p.dev_err, p.timeout_ns)) break;
+        uint8_t *sa = smem + s * C::STAGE_BYTES;
+        uint8_t *sb = sa + C::A_BYTES;
+        uint8_t *sc = sb + C::B_BYTES;
+        if (it < n_main) {
+          const int k0 = (kb_begin + it) * 64;
+          mbar_arrive_expect_tx(&full[s], C::A_BYTES + C::C_BYTES);
+          tma_load_2d(sa, &map_a, &full[s], k0, m0);
+          if (C::BMODE == B_DQ_K)
+            tma_load_2d(sc, &map_codes, &full[s], k0 / 2, nh0);  // [128 W rows x 32 B]
+          else
+            tma_load_2d(sc, &map_codes, &full[s], nh0 / 2, k0);  // [64 W rows x 64 B], 64-B swizzle
+        } else {
+          const int r0 = (it - n_main) * 64;
+          mbar_arrive_expect_tx(&full[s], C::A_BYTES + C::B_BYTES);
+          tma_load_2d(sa, &map_a2, &full[s], r0, m0);
+          if (C::LORA == LORA_B2_MN) {
+            tma_load_2d(sb, &map_b2, &full[s], nh0, r0);
+            tma_load_2d(sb + 8192, &map_b2, &full[s], nh0 + 64, r0);
+          } else {
+            tma_load_2d(sb, &map_b2, &full[s], r0, nh0);
+          }
+        }
+        issued = it + 1;
+      }
+      for (int it = issued - C::STAGES < 0 ? 0 : issued - C::STAGES; it < issued; ++it) {
+        int dummy = 0;
+        mbar_wait_bounded(&full[it % C::STAGES], (it / C::STAGES) & 1, &dummy, nullptr, kDrainNs);
+      }
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ pair MMA issuer (leader)
+    if (leader && lane == 0) {
+      constexpr uint32_t idesc_main = idesc_bf16(256, 256, false, C::B_MN);
+      constexpr uint32_t idesc_lora = idesc_bf16(256, 256, false, C::LORA == LORA_B2_MN);
+      for (int it = 0; it < n_total; ++it) {
+        const int s = it % C::STAGES;
+        const uint32_t ph = (it / C::STAGES) & 1;
+        const bool main = it < n_main;
+        if (!mbar_wait_cluster_bounded(&ready[s], ph, abort_flag, p.dev_err, p.timeout_ns)) break;
+        tc_fence_after();
+        const uint32_t a_base = smem_base + s * C::STAGE_BYTES;
+        const uint32_t b_base = a_base + C::A_BYTES;
+        int ksteps = 4;
+        if (!main) {
+          const int rem = p.lora_r - (it - n_main) * 64;
+          ksteps = rem >= 64 ? 4 : (rem + 15) / 16;
+        }
+        const bool b_mn = main ? C::B_MN : (C::LORA == LORA_B2_MN);
+        for (int kk = 0; kk < ksteps; ++kk) {
+          const uint64_t ad = smem_desc_sw128(a_base + kk * 32, 16, 1024);
+          const uint64_t bd = b_mn ? smem_desc_sw128(b_base + kk * 2048, 8192, 1024)
+                                   : smem_desc_sw128(b_base + kk * 32, 16, 1024);
+          mma_bf16_ss_pair(tmem_acc, ad, bd, main ? idesc_main : idesc_lora, (it > 0 || kk > 0) ? 1u : 0u);
+        }
+        mma_commit_pair_mc(&empty[s], 3);
+      }
+      mma_commit_pair_mc(acc_full, 3);
+    }
+  } else {
+    // ------------------------------------------------------------ dequant groups
+    const int g = (warp - 2) >> 2;                    // group 0: warps 2..5, group 1: warps 6..9
+    const int t = ((warp - 2) & 3) * 32 + lane;       // 0..127
+    const float mu = *p.mean;
+    const uint32_t ready_leader = mapa_shared(smem_u32(&ready[0]), 0);
+    for (int it = g; it < n_total; it += 2) {
+      const int s = it % C::STAGES;
+      const uint32_t ph = (it / C::STAGES) & 1;
+      const bool main = it < n_main;
+      const int kb = kb_begin + it;
+      int wrow = 0, wblk = 0;
+      if (C::BMODE == B_DQ_K) {
+        wrow = nh0 + t;
+        wblk = kb;
+      } else {
+        wrow = kb * 64 + (t & 63);
+        wblk = nh0 / 64 + (t >> 6);
+      }
+      float c2h = 0.f;
+      if (main && wrow < p.w_rows && wblk < p.w_kblocks) {
+        const int64_t b = static_cast<int64_t>(wrow) * p.w_kblocks + wblk;
+        c2h = reconstruct_c2(__ldg(p.c2q + b), __ldg(p.c1 + (b >> 8)), mu);
+      }
+      const bool ok = mbar_wait_bounded(&full[s], ph, abort_flag, p.dev_err, p.timeout_ns);
+      if (!__all_sync(0xFFFFFFFFu, ok)) break;
+      if (main) {
+        const uint32_t stage = smem_base + s * C::STAGE_BYTES;
+        const uint32_t cbase = stage + C::A_BYTES + C::B_BYTES;
+        uint32_t w[8];
+        uint32_t obase;
+        int swz;
+        if (C::BMODE == B_DQ_K) {
+          // row t: 32 bytes; threads 4..7 of each 8-thread phase read the upper half first
+          const uint32_t first = ((t >> 2) & 1) << 4;
+          uint32_t a0, a1, a2, a3, b0, b1, b2, b3;
+          ld_shared_v4(cbase + t * 32 + first, a0, a1, a2, a3);
+          ld_shared_v4(cbase + t * 32 + (16 - first), b0, b1, b2, b3);
+          const bool sw = first != 0;
+          w[0] = sw ? b0 : a0; w[1] = sw ? b1 : a1; w[2] = sw ? b2 : a2; w[3] = sw ? b3 : a3;
+          w[4] = sw ? a0 : b0; w[5] = sw ? a1 : b1; w[6] = sw ? a2 : b2; w[7] = sw ? a3 : b3;
+          obase = stage + C::A_BYTES + t * 128;
+          swz = t & 7;
+        } else {
+          const int r = t & 63, j = t >> 6;
+          const uint32_t x = (r >> 1) & 3;  // 64-byte TMA swizzle of the code tile
+          ld_shared_v4(cbase + r * 64 + ((((2 * j) ^ x) & 3) << 4), w[0], w[1], w[2], w[3]);
+          ld_shared_v4(cbase + r * 64 + ((((2 * j + 1) ^ x) & 3) << 4), w[4], w[5], w[6], w[7]);
+          obase = stage + C::A_BYTES + j * 8192 + r * 128;
+          swz = r & 7;
+        }
+        const BlockLut lut = make_lut(c2h, p.lv);
+#pragma unroll
+        for (int c = 0; c < 8; ++c) {
+          uint32_t o[4];
+          decode8(w[c], lut, o);
+          st_shared_v4(obase + ((c ^ swz) << 4), o[0], o[1], o[2], o[3]);
+        }
+        fence_proxy_async_smem();
+      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive_cluster(ready_leader + s * 8);
+    }
+    // ------------------------------------------------------------ epilogue (warps 2..5)
+    if (warp < 6) {
+      const bool got = mbar_wait_cluster_bounded(acc_full, 0, abort_flag, p.dev_err, p.timeout_ns);
+      if (__all_sync(0xFFFFFFFFu, got) && !*abort_flag) {
+        tc_fence_after();
+        const int q = warp & 3;
+        const int row = m0 + q * 32 + lane;
+        for (int c0 = 0; c0 < C::BN; c0 += 32) {
+          uint32_t v[32];
+          tmem_ld32(tmem_acc + (static_cast<uint32_t>(q * 32) << 16) + c0, v);
+          tmem_ld_wait();
+          const int col = n0 + c0;
+          if (row < p.rows && col < p.cols) {
+            if (C::OUT == OUT_BF16) {
+              uint16_t *o = reinterpret_cast<uint16_t *>(p.out) + static_cast<int64_t>(row) * p.ld_out + col;
+#pragma unroll
+              for (int gq = 0; gq < 4; ++gq) {
+                if (col + 8 * gq + 8 <= p.cols) {
+                  uint4 pk;
+                  pk.x = pack_bf16x2(__uint_as_float(v[8 * gq + 0]), __uint_as_float(v[8 * gq + 1]));
+                  pk.y = pack_bf16x2(__uint_as_float(v[8 * gq + 2]), __uint_as_float(v[8 * gq + 3]));
+                  pk.z = pack_bf16x2(__uint_as_float(v[8 * gq + 4]), __uint_as_float(v[8 * gq + 5]));
+                  pk.w = pack_bf16x2(__uint_as_float(v[8 * gq + 6]), __uint_as_float(v[8 * gq + 7]));
+                  *reinterpret_cast<uint4 *>(o + 8 * gq) = pk;
+                }
+              }
+            } else {
+              float *o = reinterpret_cast<float *>(p.out) + static_cast<int64_t>(split) * p.split_stride +
+                         static_cast<int64_t>(row) * p.ld_out + col;
+#pragma unroll
+              for (int gq = 0; gq < 8; ++gq) {
+                if (col + 4 * gq + 4 <= p.cols)
+                  *reinterpret_cast<float4 *>(o + 4 * gq) =
+                      make_float4(__uint_as_float(v[4 * gq]), __uint_as_float(v[4 * gq + 1]),
+                                  __uint_as_float(v[4 * gq + 2]), __uint_as_float(v[4 * gq + 3]));
+              }
+            }
+          }
+        }
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1 && leader && lane == 0 && *abort_flag) {
+    int dummy = 0;  // no pair MMA may still be running when TMEM is released
+    mbar_wait_cluster_bounded(acc_full, 0, &dummy, nullptr, kDrainNs);
+  }
+  cluster_sync();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc_pair(tmem_acc, C::TMEM_COLS);
+  }
+}
+
+}  // namespace qlora

@@ -18,6 +18,7 @@
 #include <cuda.h>
 #include <cuda_runtime.h>
 #include "gemm.cuh"
+#include "gemm_pair.cuh"
 #include "internal.h"
 #include "linear_plan.h"
 
@@ -50,6 +51,25 @@ static cudaError_t launch(dim3 grid, const TmaMaps &m, const GemmParams &p, cuda
   cudaError_t e = prepare<C>();
   if (e != cudaSuccess) return e;
   gemm_kernel<C><<<grid, C::NUM_THREADS, C::SMEM_BYTES, st>>>(m.a, m.b, m.a2, m.b2, p);
+  count_launches(1);
+  return cudaGetLastError();
+}
+
+using PairFwd = PairCfg<6, B_DQ_K, LORA_B2_MN, OUT_BF16>;
+using PairFwdSplit = PairCfg<6, B_DQ_K, LORA_B2_MN, OUT_F32>;
+using PairBwd = PairCfg<6, B_DQ_MN, LORA_B2_K, OUT_BF16>;
+using PairBwdSplit = PairCfg<6, B_DQ_MN, LORA_B2_K, OUT_F32>;
+
+template <class C>
+static cudaError_t launch_pair(dim3 grid, const TmaMaps &m, const GemmParams &p, cudaStream_t st) {
+  static bool prepared = false;
+  if (!prepared) {
+    cudaError_t e = cudaFuncSetAttribute(gemm_pair_kernel<C>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         C::SMEM_BYTES);
+    if (e != cudaSuccess) return e;
+    prepared = true;
+  }
+  gemm_pair_kernel<C><<<grid, C::NUM_THREADS, C::SMEM_BYTES, st>>>(m.a, m.b, m.a2, m.b2, p);
   count_launches(1);
   return cudaGetLastError();
 }
@@ -198,6 +218,59 @@ static cudaError_t run_skinny(SkinnyKind kind, const LaunchCtx &c, const SplitPl
   return launch_skinny(kind, rpad, grid, maps, p, c.stream);
 }
 
+// ---------------------------------------------------------------- fused dequant GEMM
+// fwd: D[M x N] = X·W_hatᵀ + sT·B       (W-side operand K-major: rows of W)
+// bwd: D[M x K] = dY·W_hat + sU·Aᵀ      (W-side operand MN-major: columns of W)
+// `pair` selects the CTA-pair kernel (256-token tiles); otherwise one CTA per
+// 128-token tile.  With sp.splits > 1 the K range is split and float32 partials
+// go to `part` before a fixed-order reduction.
+static cudaError_t run_fused(bool fwd, const LaunchCtx &c, const qlora_nf4_weight &w, const uint16_t *act, int64_t M,
+                             const uint16_t *lora_a, const uint16_t *lora_b, int r, uint16_t *out, bool pair,
+                             const SplitPlan &sp, float *part, cudaEvent_t ev0, cudaEvent_t ev1) {
+  cudaError_t e;
+  const int N = static_cast<int>(w.N), K = static_cast<int>(w.K);
+  const int n_out = fwd ? N : K;
+  const int red = fwd ? K : N;
+  TmaMaps m;
+  bool ok = map_bf16_kmajor(&m.a, act, red, M, 128) && map_bf16_kmajor(&m.a2, lora_a, r, M, 128);
+  if (fwd) {
+    ok = ok && map_codes(&m.b, w.codes, N, K, 32, pair ? 128 : 256, false) && map_bf16_mn(&m.b2, lora_b, N, r);
+  } else {
+    ok = ok && (pair ? map_codes(&m.b, w.codes, N, K, 64, 64, true) : map_codes(&m.b, w.codes, N, K, 128, 64, false)) &&
+         map_bf16_kmajor(&m.b2, lora_b, r, K, pair ? 128 : 256);
+  }
+  if (!ok) return cudaErrorInvalidValue;
+  GemmParams p = base_params(c);
+  p.rows = static_cast<int>(M);
+  p.cols = n_out;
+  p.k_iters = sp.k_iters;
+  p.k_iters_total = sp.k_iters_total;
+  p.lora_r = r;
+  p.c2q = w.c2q;
+  p.c1 = w.c1;
+  p.mean = w.mean;
+  p.w_rows = N;
+  p.w_kblocks = K / 64;
+  p.ld_out = n_out;
+  const bool split = sp.splits > 1;
+  p.out = split ? static_cast<void *>(part) : static_cast<void *>(out);
+  p.split_stride = M * n_out;
+  const unsigned gx = pair ? static_cast<unsigned>(2 * ((M + 255) / 256)) : static_cast<unsigned>((M + 127) / 128);
+  dim3 grid(gx, static_cast<unsigned>((n_out + 255) / 256), static_cast<unsigned>(sp.splits));
+  if (ev0) cudaEventRecord(ev0, c.stream);
+  if (pair) {
+    if (fwd) e = split ? launch_pair<PairFwdSplit>(grid, m, p, c.stream) : launch_pair<PairFwd>(grid, m, p, c.stream);
+    else e = split ? launch_pair<PairBwdSplit>(grid, m, p, c.stream) : launch_pair<PairBwd>(grid, m, p, c.stream);
+  } else {
+    if (fwd) e = split ? launch<CfgFwdSplit>(grid, m, p, c.stream) : launch<CfgFwd>(grid, m, p, c.stream);
+    else e = split ? launch<CfgBwdSplit>(grid, m, p, c.stream) : launch<CfgBwd>(grid, m, p, c.stream);
+  }
+  if (e != cudaSuccess) return e;
+  if (ev1) cudaEventRecord(ev1, c.stream);
+  if (split) return finalize_bf16(part, sp.splits, M * n_out, M, n_out, n_out, 1.0f, out, n_out, c.stream);
+  return cudaSuccess;
+}
+
 // ---------------------------------------------------------------- forward
 cudaError_t run_forward(const LaunchCtx &c, const qlora_nf4_weight &w, const uint16_t *X, int64_t M,
                         const uint16_t *A, const uint16_t *B, int r, float s, uint16_t *Y, uint16_t *T_save,
@@ -218,39 +291,11 @@ cudaError_t run_forward(const LaunchCtx &c, const qlora_nf4_weight &w, const uin
   }
   // Y = X·W_hatᵀ + sT·B
   {
-    TmaMaps m;
-    if (!map_bf16_kmajor(&m.a, X, K, M, 128) || !map_codes(&m.b, w.codes, N, K, 32, 256) ||
-        !map_bf16_kmajor(&m.a2, sT, r, M, 128) || !map_bf16_mn(&m.b2, B, N, r))
-      return cudaErrorInvalidValue;
-    GemmParams p = base_params(c);
-    p.rows = static_cast<int>(M);
-    p.cols = N;
-    p.k_iters = pl.sp_main.k_iters;
-    p.k_iters_total = pl.sp_main.k_iters_total;
-    p.lora_r = r;
-    p.c2q = w.c2q;
-    p.c1 = w.c1;
-    p.mean = w.mean;
-    p.w_rows = N;
-    p.w_kblocks = K / 64;
-    dim3 grid(static_cast<unsigned>((M + 127) / 128), static_cast<unsigned>((N + 255) / 256),
-              static_cast<unsigned>(pl.sp_main.splits));
     const TimingHooks &hk = timing_hooks();
-    if (hk.fwd_begin) cudaEventRecord(hk.fwd_begin, c.stream);
-    if (pl.sp_main.splits == 1) {
-      p.out = Y;
-      p.ld_out = N;
-      if ((e = launch<CfgFwd>(grid, m, p, c.stream)) != cudaSuccess) return e;
-      if (hk.fwd_end) cudaEventRecord(hk.fwd_end, c.stream);
-    } else {
-      float *part = reinterpret_cast<float *>(ws + pl.off_main_part);
-      p.out = part;
-      p.ld_out = N;
-      p.split_stride = M * N;
-      if ((e = launch<CfgFwdSplit>(grid, m, p, c.stream)) != cudaSuccess) return e;
-      if (hk.fwd_end) cudaEventRecord(hk.fwd_end, c.stream);
-      if ((e = finalize_bf16(part, pl.sp_main.splits, M * N, M, N, N, 1.0f, Y, N, c.stream)) != cudaSuccess) return e;
-    }
+    float *part = reinterpret_cast<float *>(ws + pl.off_main_part);
+    if ((e = run_fused(true, c, w, X, M, sT, B, r, Y, pl.pair_main, pl.sp_main, part, hk.fwd_begin, hk.fwd_end)) !=
+        cudaSuccess)
+      return e;
   }
   return cudaSuccess;
 }
@@ -290,39 +335,11 @@ cudaError_t run_backward(const LaunchCtx &c, const qlora_nf4_weight &w, const ui
   }
   // dX = dY·W_hat + sU·Aᵀ
   if (dX) {
-    TmaMaps m;
-    if (!map_bf16_kmajor(&m.a, dY, N, M, 128) || !map_codes(&m.b, w.codes, N, K, 128, 64) ||
-        !map_bf16_kmajor(&m.a2, sU, r, M, 128) || !map_bf16_kmajor(&m.b2, A, r, K, 256))
-      return cudaErrorInvalidValue;
-    GemmParams p = base_params(c);
-    p.rows = static_cast<int>(M);
-    p.cols = K;
-    p.k_iters = pl.sp_dx.k_iters;
-    p.k_iters_total = pl.sp_dx.k_iters_total;
-    p.lora_r = r;
-    p.c2q = w.c2q;
-    p.c1 = w.c1;
-    p.mean = w.mean;
-    p.w_rows = N;
-    p.w_kblocks = K / 64;
-    dim3 grid(static_cast<unsigned>((M + 127) / 128), static_cast<unsigned>((K + 255) / 256),
-              static_cast<unsigned>(pl.sp_dx.splits));
     const TimingHooks &hk = timing_hooks();
-    if (hk.bwd_begin) cudaEventRecord(hk.bwd_begin, c.stream);
-    if (pl.sp_dx.splits == 1) {
-      p.out = dX;
-      p.ld_out = K;
-      if ((e = launch<CfgBwd>(grid, m, p, c.stream)) != cudaSuccess) return e;
-      if (hk.bwd_end) cudaEventRecord(hk.bwd_end, c.stream);
-    } else {
-      float *part = reinterpret_cast<float *>(ws + pl.off_main_part);
-      p.out = part;
-      p.ld_out = K;
-      p.split_stride = M * K;
-      if ((e = launch<CfgBwdSplit>(grid, m, p, c.stream)) != cudaSuccess) return e;
-      if (hk.bwd_end) cudaEventRecord(hk.bwd_end, c.stream);
-      if ((e = finalize_bf16(part, pl.sp_dx.splits, M * K, M, K, K, 1.0f, dX, K, c.stream)) != cudaSuccess) return e;
-    }
+    float *part = reinterpret_cast<float *>(ws + pl.off_main_part);
+    if ((e = run_fused(false, c, w, dY, M, sU, A, r, dX, pl.pair_dx, pl.sp_dx, part, hk.bwd_begin, hk.bwd_end)) !=
+        cudaSuccess)
+      return e;
   }
   // dA = Xᵀ·sU : D[K x r] (A-op Xᵀ: X [M,K] MN-major; B-op sUᵀ: sU [M,r] MN-major)
   {
