@@ -10,17 +10,20 @@
 // a one-CTA 128 x 256 tile this halves the dequantisation work per flop and the
 // W-side operand bytes each SM stages.
 //
-// Roles per CTA (320 threads):
+// Roles per CTA (576 threads):
 //   warp 0      TMA producer (own activation half + own packed-code half, or
 //               the LoRA operand halves) into a STAGES-deep ring; local
 //               full[] barriers.
 //   warp 1      TMEM allocation (pair); in the leader, the MMA issuer: waits
 //               ready[s] (8 warp arrivals: 4 per CTA), issues 4 pair MMAs,
 //               commits empty[s] to both CTAs (multicast).
-//   warps 2..9  two dequant groups of 4 warps taking alternate stages: wait the
-//               local full[s], expand 128 rows x 64 codes to bf16 in the
-//               swizzled UMMA layout, fence to the async proxy, arrive on the
-//               leader's ready[s].  Warps 2..5 then run the epilogue.
+//   warps 2..17 four dequant groups of 4 warps taking every 4th stage (so the
+//               proxy fence and load latency of one stage overlap the work of
+//               the next three): wait the local full[s], expand 128 rows x 64
+//               codes to bf16 in the swizzled UMMA layout, fence to the async
+//               proxy, arrive on the leader's ready[s].  The block constants of
+//               a group's next stage are fetched one iteration ahead.  Warps
+//               2..5 then run the epilogue.
 // Shared-memory bank use: K-major code rows are read in an order that gives
 // the 8 threads of each 128-bit phase distinct banks; MN-major code tiles are
 // staged with the TMA 64-byte swizzle for the same reason.
@@ -43,7 +46,8 @@ struct PairCfg {
   static constexpr int B_BYTES = 128 * 64 * 2;
   static constexpr int C_BYTES = 4096;
   static constexpr int STAGE_BYTES = A_BYTES + B_BYTES + C_BYTES;
-  static constexpr int NUM_THREADS = 320;
+  static constexpr int DQ_GROUPS = 4;  // groups of 4 warps taking every 4th stage
+  static constexpr int NUM_THREADS = 64 + 128 * DQ_GROUPS;
   static constexpr int TMEM_COLS = 256;
   static constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + 256 + 1024;
   static_assert(BMODE == B_DQ_K || BMODE == B_DQ_MN, "pair kernel dequantises its W-side operand");
@@ -176,16 +180,17 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(C::NUM_THREADS, 1)
     }
   } else {
     // ------------------------------------------------------------ dequant groups
-    const int g = (warp - 2) >> 2;                    // group 0: warps 2..5, group 1: warps 6..9
+    const int g = (warp - 2) >> 2;                    // dequant group
     const int t = ((warp - 2) & 3) * 32 + lane;       // 0..127
     const float mu = *p.mean;
     const uint32_t ready_leader = mapa_shared(smem_u32(&ready[0]), 0);
-    for (int it = g; it < n_total; it += 2) {
-      const int s = it % C::STAGES;
-      const uint32_t ph = (it / C::STAGES) & 1;
-      const bool main = it < n_main;
+    // block constant of this thread's (row, block) at stage `it` (raw E4M3 byte + group scale)
+    auto fetch = [&](int it, uint32_t &e, float &sg) {
+      e = 0;
+      sg = 0.f;
+      if (it >= n_main) return;
       const int kb = kb_begin + it;
-      int wrow = 0, wblk = 0;
+      int wrow, wblk;
       if (C::BMODE == B_DQ_K) {
         wrow = nh0 + t;
         wblk = kb;
@@ -193,11 +198,25 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(C::NUM_THREADS, 1)
         wrow = kb * 64 + (t & 63);
         wblk = nh0 / 64 + (t >> 6);
       }
-      float c2h = 0.f;
-      if (main && wrow < p.w_rows && wblk < p.w_kblocks) {
+      if (wrow < p.w_rows && wblk < p.w_kblocks) {
         const int64_t b = static_cast<int64_t>(wrow) * p.w_kblocks + wblk;
-        c2h = reconstruct_c2(__ldg(p.c2q + b), __ldg(p.c1 + (b >> 8)), mu);
+        e = __ldg(p.c2q + b);
+        sg = __ldg(p.c1 + (b >> 8));
       }
+    };
+    uint32_t e_cur;
+    float s_cur;
+    fetch(g, e_cur, s_cur);
+    for (int it = g; it < n_total; it += C::DQ_GROUPS) {
+      const int s = it % C::STAGES;
+      const uint32_t ph = (it / C::STAGES) & 1;
+      const bool main = it < n_main;
+      uint32_t e_nxt;
+      float s_nxt;
+      fetch(it + C::DQ_GROUPS, e_nxt, s_nxt);
+      const float c2h = main ? reconstruct_c2(e_cur, s_cur, mu) : 0.f;
+      e_cur = e_nxt;
+      s_cur = s_nxt;
       const bool ok = mbar_wait_bounded(&full[s], ph, abort_flag, p.dev_err, p.timeout_ns);
       if (!__all_sync(0xFFFFFFFFu, ok)) break;
       if (main) {
