@@ -146,12 +146,12 @@ LinearPlan make_plan(int op, int64_t M, int64_t N, int64_t K, int r, int num_sms
   pl.off_t_part = take(static_cast<size_t>(pl.sp_t.splits) * M * pl.rpad * 4);
   if (op == QLORA_OP_FORWARD) {
     pl.pair_main = M > 128;
-    pl.sp_main = choose((pl.pair_main ? 2 * ((M + 255) / 256) : mt) * ((N + 255) / 256), K / 64, num_sms, 4);
+    pl.sp_main = choose((pl.pair_main ? 2 * ((M + 511) / 512) : mt) * ((N + 255) / 256), K / 64, num_sms, 4);
     if (pl.sp_main.splits > 1) pl.off_main_part = take(static_cast<size_t>(pl.sp_main.splits) * M * N * 4);
   } else {
     pl.sp_u = choose(mt, (N + 63) / 64, 2 * num_sms, 2);
     pl.pair_dx = M > 128;
-    pl.sp_dx = choose((pl.pair_dx ? 2 * ((M + 255) / 256) : mt) * ((K + 255) / 256), (N + 63) / 64, num_sms, 4);
+    pl.sp_dx = choose((pl.pair_dx ? 2 * ((M + 511) / 512) : mt) * ((K + 255) / 256), (N + 63) / 64, num_sms, 4);
     pl.sp_da = choose((K + 127) / 128, (M + 63) / 64, 2 * num_sms, 2);
     pl.sp_db = choose((N + 127) / 128, (M + 63) / 64, 2 * num_sms, 2);
     pl.off_sU = take(static_cast<size_t>(M) * r * 2);

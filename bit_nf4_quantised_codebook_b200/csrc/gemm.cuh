@@ -56,6 +56,8 @@ struct GemmParams {
   int64_t split_stride;  // elements between split partials (OUT_F32)
   int *dev_err;
   unsigned long long timeout_ns;
+  uint32_t k_shr16;  // 2^16 (a right shift by 16 done as a high-half multiply)
+  uint32_t k_shr1;   // 2^31 (a right shift by 1 likewise)
 };
 
 template <int BN_, int STAGES_, bool A_MN_, int BMODE_, int LORA_, int OUT_>

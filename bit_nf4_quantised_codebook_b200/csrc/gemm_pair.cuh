@@ -1,14 +1,16 @@
 // gemm_pair.cuh — the fused dequant GEMM on a CTA pair (cluster of 2, tcgen05
-// cta_group::2): one 256 x 256 output tile per pair.
+// cta_group::2): one (256·MSUB) x 256 output tile per pair.
 //
-//   D[256 tokens x 256] = sum_k Aop[256 x k] · W_hat-side[256 x k]ᵀ  (+ LoRA tail)
+//   D[256·MSUB tokens x 256] = sum_k Aop · W_hat-sideᵀ  (+ LoRA tail)
 //
-// Each CTA of the pair stages its own 128 token rows of the activation (TMA)
+// Each CTA of the pair stages its own 128·MSUB token rows of the activation (TMA)
 // and dequantises its own 128 rows of the W-side operand; the leader CTA issues
 // the pair MMA, which reads both CTAs' shared memory at the same offsets and
-// writes each CTA's 128 x 256 accumulator slice into that CTA's TMEM.  Against
-// a one-CTA 128 x 256 tile this halves the dequantisation work per flop and the
-// W-side operand bytes each SM stages.
+// writes each CTA's 128 x 256 accumulator slice into that CTA's TMEM; with
+// MSUB = 2 every dequantised W tile feeds two such MMAs (two accumulators, all
+// 512 TMEM columns).  Against a one-CTA 128 x 256 tile this cuts the
+// dequantisation work per flop by 2·MSUB and the W-side operand bytes each SM
+// stages by 2.
 //
 // Roles per CTA (576 threads):
 //   warp 0      TMA producer (own activation half + own packed-code half, or
@@ -22,8 +24,8 @@
 //               the next three): wait the local full[s], expand 128 rows x 64
 //               codes to bf16 in the swizzled UMMA layout, fence to the async
 //               proxy, arrive on the leader's ready[s].  The block constants of
-//               a group's next stage are fetched one iteration ahead.  Warps
-//               2..5 then run the epilogue.
+//               a group's next stage are fetched one iteration ahead.  All
+//               16 then run the epilogue.
 // Shared-memory bank use: K-major code rows are read in an order that gives
 // the 8 threads of each 128-bit phase distinct banks; MN-major code tiles are
 // staged with the TMA 64-byte swizzle for the same reason.
@@ -34,21 +36,22 @@
 
 namespace qlora {
 
-template <int STAGES_, int BMODE_, int LORA_, int OUT_>
+template <int STAGES_, int BMODE_, int LORA_, int OUT_, int MSUB_>
 struct PairCfg {
   static constexpr int STAGES = STAGES_;
+  static constexpr int MSUB = MSUB_;  // 128-token sub-tiles per CTA sharing one dequantised W tile
   static constexpr int BMODE = BMODE_;
   static constexpr int LORA = LORA_;
   static constexpr int OUT = OUT_;
   static constexpr int BN = 256;  // pair N
   static constexpr bool B_MN = BMODE == B_DQ_MN;
-  static constexpr int A_BYTES = 128 * 64 * 2;
+  static constexpr int A_BYTES = MSUB * 128 * 64 * 2;
   static constexpr int B_BYTES = 128 * 64 * 2;
   static constexpr int C_BYTES = 4096;
   static constexpr int STAGE_BYTES = A_BYTES + B_BYTES + C_BYTES;
   static constexpr int DQ_GROUPS = 4;  // groups of 4 warps taking every 4th stage
   static constexpr int NUM_THREADS = 64 + 128 * DQ_GROUPS;
-  static constexpr int TMEM_COLS = 256;
+  static constexpr int TMEM_COLS = 256 * MSUB;
   static constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + 256 + 1024;
   static_assert(BMODE == B_DQ_K || BMODE == B_DQ_MN, "pair kernel dequantises its W-side operand");
   static_assert(STAGE_BYTES % 1024 == 0, "swizzle atoms need 1 KiB alignment");
@@ -73,7 +76,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(C::NUM_THREADS, 1)
   const int lane = threadIdx.x & 31;
   const uint32_t rank = cluster_ctarank();
   const bool leader = rank == 0;
-  const int m0 = blockIdx.x * 128;            // this CTA's token rows
+  const int m0 = blockIdx.x * 128 * C::MSUB;  // this CTA's token rows (MSUB sub-tiles of 128)
   const int n0 = blockIdx.y * C::BN;          // the pair's W-side tile
   const int nh0 = n0 + 128 * static_cast<int>(rank);  // this CTA's half of it
   const int split = blockIdx.z;
@@ -126,7 +129,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(C::NUM_THREADS, 1)
         if (it < n_main) {
           const int k0 = (kb_begin + it) * 64;
           mbar_arrive_expect_tx(&full[s], C::A_BYTES + C::C_BYTES);
-          tma_load_2d(sa, &map_a, &full[s], k0, m0);
+#pragma unroll
+          for (int i = 0; i < C::MSUB; ++i) tma_load_2d(sa + i * 16384, &map_a, &full[s], k0, m0 + 128 * i);
           if (C::BMODE == B_DQ_K)
             tma_load_2d(sc, &map_codes, &full[s], k0 / 2, nh0);  // [128 W rows x 32 B]
           else
@@ -134,7 +138,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(C::NUM_THREADS, 1)
         } else {
           const int r0 = (it - n_main) * 64;
           mbar_arrive_expect_tx(&full[s], C::A_BYTES + C::B_BYTES);
-          tma_load_2d(sa, &map_a2, &full[s], r0, m0);
+#pragma unroll
+          for (int i = 0; i < C::MSUB; ++i) tma_load_2d(sa + i * 16384, &map_a2, &full[s], r0, m0 + 128 * i);
           if (C::LORA == LORA_B2_MN) {
             tma_load_2d(sb, &map_b2, &full[s], nh0, r0);
             tma_load_2d(sb + 8192, &map_b2, &full[s], nh0 + 64, r0);
@@ -169,10 +174,14 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(C::NUM_THREADS, 1)
         }
         const bool b_mn = main ? C::B_MN : (C::LORA == LORA_B2_MN);
         for (int kk = 0; kk < ksteps; ++kk) {
-          const uint64_t ad = smem_desc_sw128(a_base + kk * 32, 16, 1024);
           const uint64_t bd = b_mn ? smem_desc_sw128(b_base + kk * 2048, 8192, 1024)
                                    : smem_desc_sw128(b_base + kk * 32, 16, 1024);
-          mma_bf16_ss_pair(tmem_acc, ad, bd, main ? idesc_main : idesc_lora, (it > 0 || kk > 0) ? 1u : 0u);
+#pragma unroll
+          for (int i = 0; i < C::MSUB; ++i) {
+            const uint64_t ad = smem_desc_sw128(a_base + i * 16384 + kk * 32, 16, 1024);
+            mma_bf16_ss_pair(tmem_acc + 256 * i, ad, bd, main ? idesc_main : idesc_lora,
+                             (it > 0 || kk > 0) ? 1u : 0u);
+          }
         }
         mma_commit_pair_mc(&empty[s], 3);
       }
@@ -245,52 +254,60 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(C::NUM_THREADS, 1)
           swz = r & 7;
         }
         const BlockLut lut = make_lut(c2h, p.lv);
+        const uint32_t sbase = obase | (static_cast<uint32_t>(swz) << 4);  // obase is 128-byte aligned
 #pragma unroll
         for (int c = 0; c < 8; ++c) {
           uint32_t o[4];
-          decode8(w[c], lut, o);
-          st_shared_v4(obase + ((c ^ swz) << 4), o[0], o[1], o[2], o[3]);
+          decode8(w[c], lut, o, p.k_shr16, p.k_shr1);
+          st_shared_v4(sbase ^ (static_cast<uint32_t>(c) << 4), o[0], o[1], o[2], o[3]);
         }
         fence_proxy_async_smem();
       }
       __syncwarp();
       if (lane == 0) mbar_arrive_cluster(ready_leader + s * 8);
     }
-    // ------------------------------------------------------------ epilogue (warps 2..5)
-    if (warp < 6) {
+    // ------------------------------------------------------------ epilogue (all dequant warps)
+    // warp w reads TMEM lane quadrant (w & 3) and a 64-column slice ((w - 2) >> 2) of
+    // every 256-column accumulator.
+    {
       const bool got = mbar_wait_cluster_bounded(acc_full, 0, abort_flag, p.dev_err, p.timeout_ns);
       if (__all_sync(0xFFFFFFFFu, got) && !*abort_flag) {
         tc_fence_after();
         const int q = warp & 3;
-        const int row = m0 + q * 32 + lane;
-        for (int c0 = 0; c0 < C::BN; c0 += 32) {
-          uint32_t v[32];
-          tmem_ld32(tmem_acc + (static_cast<uint32_t>(q * 32) << 16) + c0, v);
-          tmem_ld_wait();
-          const int col = n0 + c0;
-          if (row < p.rows && col < p.cols) {
-            if (C::OUT == OUT_BF16) {
-              uint16_t *o = reinterpret_cast<uint16_t *>(p.out) + static_cast<int64_t>(row) * p.ld_out + col;
+        const int cg = (warp - 2) >> 2;
+#pragma unroll 1
+        for (int i = 0; i < C::MSUB; ++i) {
+          const int row = m0 + 128 * i + q * 32 + lane;
+#pragma unroll 1
+          for (int c0 = cg * 64; c0 < cg * 64 + 64; c0 += 32) {
+            uint32_t v[32];
+            tmem_ld32(tmem_acc + (static_cast<uint32_t>(q * 32) << 16) + 256 * i + c0, v);
+            tmem_ld_wait();
+            const int col = n0 + c0;
+            if (row < p.rows && col < p.cols) {
+              if (C::OUT == OUT_BF16) {
+                uint16_t *o = reinterpret_cast<uint16_t *>(p.out) + static_cast<int64_t>(row) * p.ld_out + col;
 #pragma unroll
-              for (int gq = 0; gq < 4; ++gq) {
-                if (col + 8 * gq + 8 <= p.cols) {
-                  uint4 pk;
-                  pk.x = pack_bf16x2(__uint_as_float(v[8 * gq + 0]), __uint_as_float(v[8 * gq + 1]));
-                  pk.y = pack_bf16x2(__uint_as_float(v[8 * gq + 2]), __uint_as_float(v[8 * gq + 3]));
-                  pk.z = pack_bf16x2(__uint_as_float(v[8 * gq + 4]), __uint_as_float(v[8 * gq + 5]));
-                  pk.w = pack_bf16x2(__uint_as_float(v[8 * gq + 6]), __uint_as_float(v[8 * gq + 7]));
-                  *reinterpret_cast<uint4 *>(o + 8 * gq) = pk;
+                for (int gq = 0; gq < 4; ++gq) {
+                  if (col + 8 * gq + 8 <= p.cols) {
+                    uint4 pk;
+                    pk.x = pack_bf16x2(__uint_as_float(v[8 * gq + 0]), __uint_as_float(v[8 * gq + 1]));
+                    pk.y = pack_bf16x2(__uint_as_float(v[8 * gq + 2]), __uint_as_float(v[8 * gq + 3]));
+                    pk.z = pack_bf16x2(__uint_as_float(v[8 * gq + 4]), __uint_as_float(v[8 * gq + 5]));
+                    pk.w = pack_bf16x2(__uint_as_float(v[8 * gq + 6]), __uint_as_float(v[8 * gq + 7]));
+                    *reinterpret_cast<uint4 *>(o + 8 * gq) = pk;
+                  }
                 }
-              }
-            } else {
-              float *o = reinterpret_cast<float *>(p.out) + static_cast<int64_t>(split) * p.split_stride +
-                         static_cast<int64_t>(row) * p.ld_out + col;
+              } else {
+                float *o = reinterpret_cast<float *>(p.out) + static_cast<int64_t>(split) * p.split_stride +
+                           static_cast<int64_t>(row) * p.ld_out + col;
 #pragma unroll
-              for (int gq = 0; gq < 8; ++gq) {
-                if (col + 4 * gq + 4 <= p.cols)
-                  *reinterpret_cast<float4 *>(o + 4 * gq) =
-                      make_float4(__uint_as_float(v[4 * gq]), __uint_as_float(v[4 * gq + 1]),
-                                  __uint_as_float(v[4 * gq + 2]), __uint_as_float(v[4 * gq + 3]));
+                for (int gq = 0; gq < 8; ++gq) {
+                  if (col + 4 * gq + 4 <= p.cols)
+                    *reinterpret_cast<float4 *>(o + 4 * gq) =
+                        make_float4(__uint_as_float(v[4 * gq]), __uint_as_float(v[4 * gq + 1]),
+                                    __uint_as_float(v[4 * gq + 2]), __uint_as_float(v[4 * gq + 3]));
+                }
               }
             }
           }

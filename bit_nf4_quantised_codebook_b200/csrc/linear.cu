@@ -55,10 +55,11 @@ static cudaError_t launch(dim3 grid, const TmaMaps &m, const GemmParams &p, cuda
   return cudaGetLastError();
 }
 
-using PairFwd = PairCfg<6, B_DQ_K, LORA_B2_MN, OUT_BF16>;
-using PairFwdSplit = PairCfg<6, B_DQ_K, LORA_B2_MN, OUT_F32>;
-using PairBwd = PairCfg<6, B_DQ_MN, LORA_B2_K, OUT_BF16>;
-using PairBwdSplit = PairCfg<6, B_DQ_MN, LORA_B2_K, OUT_F32>;
+using PairFwd = PairCfg<4, B_DQ_K, LORA_B2_MN, OUT_BF16, 2>;
+using PairFwdSplit = PairCfg<4, B_DQ_K, LORA_B2_MN, OUT_F32, 2>;
+using PairBwd = PairCfg<4, B_DQ_MN, LORA_B2_K, OUT_BF16, 2>;
+using PairBwdSplit = PairCfg<4, B_DQ_MN, LORA_B2_K, OUT_F32, 2>;
+constexpr int kPairTokens = 2 * 128 * 2;  // tokens per CTA pair (2 CTAs x MSUB x 128)
 
 template <class C>
 static cudaError_t launch_pair(dim3 grid, const TmaMaps &m, const GemmParams &p, cudaStream_t st) {
@@ -199,6 +200,8 @@ static GemmParams base_params(const LaunchCtx &c) {
   p.dev_err = c.dev_err;
   p.timeout_ns = c.timeout_ns;
   p.lv = c.levels;
+  p.k_shr16 = 1u << 16;
+  p.k_shr1 = 1u << 31;
   return p;
 }
 
@@ -255,7 +258,8 @@ static cudaError_t run_fused(bool fwd, const LaunchCtx &c, const qlora_nf4_weigh
   const bool split = sp.splits > 1;
   p.out = split ? static_cast<void *>(part) : static_cast<void *>(out);
   p.split_stride = M * n_out;
-  const unsigned gx = pair ? static_cast<unsigned>(2 * ((M + 255) / 256)) : static_cast<unsigned>((M + 127) / 128);
+  const unsigned gx = pair ? static_cast<unsigned>(2 * ((M + kPairTokens - 1) / kPairTokens))
+                           : static_cast<unsigned>((M + 127) / 128);
   dim3 grid(gx, static_cast<unsigned>((n_out + 255) / 256), static_cast<unsigned>(sp.splits));
   if (ev0) cudaEventRecord(ev0, c.stream);
   if (pair) {

@@ -78,4 +78,16 @@ __device__ __forceinline__ void decode8(uint32_t w, const BlockLut &t, uint32_t 
   decode4(s7 >> 16, sm >> 16, t, o[2], o[3]);
 }
 
+// Same result; the three right shifts are done as high-half multiplies by the
+// run-time constants k16 = 2^16 and k1 = 2^31, which issue on the FMA pipe and
+// leave the integer/permute (ALU) pipe — the dequantiser's bottleneck — to the
+// byte permutes.
+__device__ __forceinline__ void decode8(uint32_t w, const BlockLut &t, uint32_t (&o)[4], uint32_t k16,
+                                        uint32_t k1) {
+  const uint32_t s7 = w & 0x77777777u;
+  const uint32_t sm = (__umulhi(w, k1) & 0x44444444u) | 0x32103210u;
+  decode4(s7, sm, t, o[0], o[1]);
+  decode4(__umulhi(s7, k16), __umulhi(sm, k16), t, o[2], o[3]);
+}
+
 }  // namespace qlora
