@@ -22,7 +22,7 @@ QLORA_DEVERR_NONFINITE, QLORA_DEVERR_TIMEOUT = 1, 2
 EXPORTED = [
     "qlora_status_string", "qlora_build_codebook", "qlora_nf4_sizes", "qlora_workspace_size",
     "qlora_quantize", "qlora_dequantize", "qlora_linear_forward", "qlora_linear_backward",
-    "qlora_kernel_launch_count", "qlora_set_timing_events",
+    "qlora_kernel_launch_count", "qlora_set_timing_events", "qlora_quantize_noalloc",
 ]
 
 
@@ -60,6 +60,7 @@ def lib() -> ctypes.CDLL:
         L.qlora_kernel_launch_count.restype = ctypes.c_uint64
         L.qlora_kernel_launch_count.argtypes = []
         L.qlora_set_timing_events.argtypes = [vp, vp, vp, vp]
+        L.qlora_quantize_noalloc.argtypes = [vp, ctypes.POINTER(_Weight), vp, vp]
         for name in EXPORTED[1:]:
             if name != "qlora_kernel_launch_count":
                 getattr(L, name).restype = i32
@@ -155,6 +156,20 @@ def qlora_quantize(W: torch.Tensor, out: NF4Weight | None = None, ws: torch.Tens
     s = out.c_struct()
     _check(lib().qlora_quantize(W.data_ptr(), ctypes.byref(s), ws.data_ptr(), ws.numel(), _ptr(dev_err),
                                 _stream()), "qlora_quantize")
+    return out
+
+
+def qlora_quantize_noalloc(W: torch.Tensor, out: NF4Weight, dev_err: torch.Tensor | None = None) -> NF4Weight:
+    """Quantise into the caller's buffers `out` without any workspace: the
+    library keeps the scratch in a static device array (N*K <= 2^26).  For
+    callers that cannot allocate device memory; see include/qlora_nf4.h."""
+    N, K = W.shape
+    _need(W, torch.bfloat16, (N, K), "W")
+    if (out.N, out.K) != (N, K):
+        raise QloraError(f"out is {out.N}x{out.K}, W is {N}x{K}")
+    s = out.c_struct()
+    _check(lib().qlora_quantize_noalloc(W.data_ptr(), ctypes.byref(s), _ptr(dev_err), _stream()),
+           "qlora_quantize_noalloc")
     return out
 
 

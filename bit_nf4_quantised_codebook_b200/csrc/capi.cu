@@ -192,6 +192,7 @@ const char *qlora_status_string(qlora_status st) {
     case QLORA_ERR_CUDA: return "CUDA error";
     case QLORA_ERR_WORKSPACE: return "workspace missing or too small";
     case QLORA_ERR_NO_DEVICE: return "current device is not sm_100";
+    case QLORA_ERR_TOO_LARGE: return "weight larger than the static scratch of qlora_quantize_noalloc (N*K <= 2^26)";
   }
   return "unknown status";
 }

@@ -64,7 +64,8 @@ typedef enum {
   QLORA_ERR_MISALIGNED = 3,        /* a device pointer is not 16-byte aligned */
   QLORA_ERR_CUDA = 4,              /* a CUDA runtime / driver call failed */
   QLORA_ERR_WORKSPACE = 5,         /* workspace missing or smaller than qlora_workspace_size() */
-  QLORA_ERR_NO_DEVICE = 6          /* the current device is not sm_100 */
+  QLORA_ERR_NO_DEVICE = 6,         /* the current device is not sm_100 */
+  QLORA_ERR_TOO_LARGE = 7          /* shape exceeds qlora_quantize_noalloc's static scratch (N*K <= 2^26) */
 } qlora_status;
 
 /* Bits OR-ed into *dev_err by kernels. */
@@ -127,6 +128,27 @@ qlora_status qlora_workspace_size(int op, int64_t M, int64_t N, int64_t K, int r
  */
 qlora_status qlora_quantize(const uint16_t *W, const qlora_nf4_weight *out, void *ws,
                             size_t ws_bytes, int *dev_err, void *stream);
+
+/*
+ * qlora_quantize_noalloc — the same quantiser (identical output bits to
+ * qlora_quantize) for callers that cannot allocate device memory: a plugin or
+ * custom-op interface that passes buffers but no allocator, or a runtime whose
+ * memory plan forbids new allocations while it runs.  No counterpart on the
+ * pages: it only changes where the scratch lives.  Instead of a caller-provided
+ * workspace it uses a static device array built into the library (about 4 MiB,
+ * held by every GPU that loads the library until the process exits), so it
+ * calls no cudaMalloc, cudaFree or allocating routine.
+ * Limit: N*K <= 2^26 (e.g. 8192 x 8192); larger weights return
+ * QLORA_ERR_TOO_LARGE and launch nothing.
+ * The first call on each device (with that device current) looks up the
+ * array's device address; make that first call before any stream capture.
+ * All calls share the array: calls that overlap on the GPU (different
+ * streams or host threads) race and give undefined results; calls ordered on
+ * one stream are safe.  The array keeps the last call's contents; nothing in it
+ * needs clearing between calls.
+ * W, out, dev_err, stream: as for qlora_quantize.
+ */
+qlora_status qlora_quantize_noalloc(const uint16_t *W, const qlora_nf4_weight *out, int *dev_err, void *stream);
 
 /*
  * qlora_dequantize — doubleDequant of §The QLoRA layer, end to end, written
