@@ -1,0 +1,69 @@
+// nf4_quant.cuh — exact normalisation and nearest-level code of one weight.
+//
+// "QLoRA: Efficient Finetuning of Quantized LLMs" (intuitivepapers.ai),
+// §Quantize in blocks / §NormalFloat: each weight is divided by its block's
+// absmax and mapped to the nearest NF4 level.  The library defines
+//   x_hat = float32(w / absmax)   (IEEE division, round to nearest even)
+//   code  = #{ i : x_hat >= t_i }  (t_i = smallest float32 above midpoint i)
+// and must reproduce both exactly.  Two cheaper, exact, steps:
+//
+// Quotient.  With y = RN(1/a) and q = RN(x·y), the residual r = x - a·q is
+// exact as one fused multiply-add, and RN(q + r·y) = RN(x/a) (Markstein's
+// correction theorem for a reciprocal within half an ulp and a quotient within
+// one ulp; P. Markstein, IBM J. Res. Dev. 34(1), 1990).  Per block the
+// reciprocal is computed once; each element then costs one multiply and two
+// fused multiply-adds.  tests/test_gpu_quotient.py checks the result against
+// CUDA's own correctly rounded division for every pair of bfloat16 inputs with
+// |x| <= a that the quantiser can meet.
+//
+// Code.  x_hat lies in [-1, 1].  Cut that range into 64 buckets of width 1/32;
+// widen each by a margin far above any rounding error of the bucket index
+// computation and far below the smallest gap between two thresholds (0.0796).
+// Each widened bucket then holds at most one threshold, so
+//   code = base[b] + (x_hat >= thr[b]),
+// with base[b] = thresholds below the widened bucket and thr[b] the one inside
+// it (+inf if none).  The 64-entry table is built per CTA from the thresholds.
+#pragma once
+#include <cstdint>
+
+namespace qlora {
+
+constexpr int kBuckets = 64;
+constexpr float kBucketScale = 32.0f;          // buckets per unit of x_hat
+constexpr float kBucketMargin = 1.0f / 1024;   // widening on each side
+
+struct CodeBucket {
+  int base;
+  float thr;
+};
+
+// RN(x / a) for finite x, a > 0 with |x| <= a, given ra = RN(1/a).
+__device__ __forceinline__ float quotient_rn(float x, float a, float ra) {
+  const float q = __fmul_rn(x, ra);
+  const float r = __fmaf_rn(-q, a, x);
+  return __fmaf_rn(r, ra, q);
+}
+
+// Fill bucket b (0..63) from the 15 thresholds.
+__device__ __forceinline__ CodeBucket make_bucket(int b, const float (&t)[15]) {
+  const float lo = static_cast<float>(b) / kBucketScale - 1.0f - kBucketMargin;
+  const float hi = static_cast<float>(b + 1) / kBucketScale - 1.0f + kBucketMargin;
+  CodeBucket e;
+  e.base = 0;
+  e.thr = __int_as_float(0x7F800000);  // +inf
+#pragma unroll
+  for (int i = 0; i < 15; ++i) {
+    if (t[i] < lo) e.base += 1;
+    else if (t[i] <= hi) e.thr = t[i];
+  }
+  return e;
+}
+
+__device__ __forceinline__ uint32_t bucket_code(float xh, const CodeBucket *tab) {
+  int b = __float2int_rd(__fmaf_rn(xh, kBucketScale, kBucketScale));
+  b = min(max(b, 0), kBuckets - 1);
+  const CodeBucket e = tab[b];
+  return static_cast<uint32_t>(e.base + (xh >= e.thr ? 1 : 0));
+}
+
+}  // namespace qlora

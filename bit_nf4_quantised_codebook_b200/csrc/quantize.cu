@@ -9,8 +9,9 @@
 //
 // Three launches, all HBM-streaming and deterministic:
 //   k_quant_blocks : one CTA per group of 256 blocks.  8 threads per block, one
-//                    16-byte load each; absmax by 3 xor-shuffles; codes by
-//                    threshold counting; nibble packing; per-group float64 sum of
+//                    16-byte load each (all eight of a thread's loads issued
+//                    first); absmax by 3 xor-shuffles; exact quotient and code
+//                    via nf4_quant.cuh; nibble packing; per-group float64 sum of
 //                    the absmax values in block order (sequential, one thread).
 //   k_mean_tree    : one CTA, power-of-two pairwise tree over the group sums.
 //   k_double_quant : one CTA per group: centred constants, group absmax, S_g,
@@ -19,6 +20,7 @@
 #include <cuda_runtime.h>
 #include "internal.h"
 #include "nf4_decode.cuh"
+#include "nf4_quant.cuh"
 
 namespace qlora {
 
@@ -35,23 +37,44 @@ __device__ __forceinline__ uint32_t nf4_code(float xh, const Nf4Thresholds &t) {
   return c;
 }
 
-__global__ void __launch_bounds__(256) k_quant_blocks(const uint16_t *__restrict__ W, int64_t nb,
+// Streaming 16-byte load that does not keep the line in L1.
+__device__ __forceinline__ uint4 ld_stream_v4(const void *p) {
+  uint4 v;
+  asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0, %1, %2, %3}, [%4];"
+               : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+               : "l"(p));
+  return v;
+}
+
+// Blocks whose absmax is at least this use the reciprocal + corrected-quotient
+// path (exact there: see nf4_quant.cuh); smaller ones divide directly.
+constexpr float kFastQuotientMinAbsmax = 7.888609052210118e-31f;  // 2^-100
+
+__global__ void __launch_bounds__(256, 2) k_quant_blocks(const uint16_t *__restrict__ W, int64_t nb,
                                                        uint8_t *__restrict__ codes, float *__restrict__ absmax,
                                                        double *__restrict__ gsum, Nf4Thresholds thr,
                                                        int *dev_err) {
   __shared__ float s_amax[256];
+  __shared__ CodeBucket s_tab[kBuckets];
+  if (threadIdx.x < kBuckets) s_tab[threadIdx.x] = make_bucket(threadIdx.x, thr.t);
   const int64_t g = blockIdx.x;
   const int part = threadIdx.x & 7;  // 8-element chunk of the block
   const int sub = threadIdx.x >> 3;  // block within the pass
+  // all eight 16-byte loads of this thread in flight at once
+  uint4 raw[8];
+#pragma unroll
+  for (int pass = 0; pass < 8; ++pass) {
+    const int64_t b = g * 256 + pass * 32 + sub;
+    raw[pass] = b < nb ? ld_stream_v4(W + b * 64 + part * 8) : make_uint4(0, 0, 0, 0);
+  }
+  __syncthreads();  // bucket table ready
   bool bad = false;
-#pragma unroll 1
+#pragma unroll
   for (int pass = 0; pass < 8; ++pass) {
     const int lb = pass * 32 + sub;
     const int64_t b = g * 256 + lb;
     const bool valid = b < nb;
-    uint4 raw = make_uint4(0, 0, 0, 0);
-    if (valid) raw = __ldg(reinterpret_cast<const uint4 *>(W + b * 64) + part);
-    const uint32_t u[4] = {raw.x, raw.y, raw.z, raw.w};
+    const uint32_t u[4] = {raw[pass].x, raw[pass].y, raw[pass].z, raw[pass].w};
     float x[8];
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
@@ -68,13 +91,24 @@ __global__ void __launch_bounds__(256) k_quant_blocks(const uint16_t *__restrict
     amax = fmaxf(amax, __shfl_xor_sync(0xFFFFFFFFu, amax, 1));
     amax = fmaxf(amax, __shfl_xor_sync(0xFFFFFFFFu, amax, 2));
     amax = fmaxf(amax, __shfl_xor_sync(0xFFFFFFFFu, amax, 4));
-    uint32_t packed = 0;
+    uint32_t packed = 0x77777777u;  // all-zero block: every code is the zero level
+    if (amax >= kFastQuotientMinAbsmax) {
+      const float ra = __frcp_rn(amax);
+      packed = 0;
 #pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      const float xa = amax == 0.f ? 0.f : __fdiv_rn(x[2 * i], amax);
-      const float xb = amax == 0.f ? 0.f : __fdiv_rn(x[2 * i + 1], amax);
-      const uint32_t byte = (nf4_code(xa, thr) << 4) | nf4_code(xb, thr);
-      packed |= byte << (8 * i);
+      for (int i = 0; i < 4; ++i) {
+        const uint32_t hi = bucket_code(quotient_rn(x[2 * i], amax, ra), s_tab);
+        const uint32_t lo = bucket_code(quotient_rn(x[2 * i + 1], amax, ra), s_tab);
+        packed |= ((hi << 4) | lo) << (8 * i);
+      }
+    } else if (amax > 0.f) {
+      packed = 0;
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const uint32_t hi = nf4_code(__fdiv_rn(x[2 * i], amax), thr);
+        const uint32_t lo = nf4_code(__fdiv_rn(x[2 * i + 1], amax), thr);
+        packed |= ((hi << 4) | lo) << (8 * i);
+      }
     }
     if (valid) {
       reinterpret_cast<uint32_t *>(codes + b * 32)[part] = packed;
@@ -92,15 +126,37 @@ __global__ void __launch_bounds__(256) k_quant_blocks(const uint16_t *__restrict
   }
 }
 
+// Pairwise tree over the power-of-two padded group sums: for h = size/2, ..., 1
+// every a[i] (i < h) becomes a[i] + a[i+h].  Levels with h >= 1024 run in global
+// memory, h = 512..32 in shared memory, h = 16..1 as warp shuffles — the same
+// additions in the same order at every level.
 __global__ void __launch_bounds__(1024) k_mean_tree(double *__restrict__ a, int64_t ng, int64_t size, int64_t nb,
                                                      float *__restrict__ mean) {
+  __shared__ double s[1024];
   for (int64_t i = ng + threadIdx.x; i < size; i += blockDim.x) a[i] = 0.0;
   __syncthreads();
-  for (int64_t h = size / 2; h >= 1; h /= 2) {
+  int64_t h = size / 2;
+  for (; h >= 1024; h /= 2) {
     for (int64_t i = threadIdx.x; i < h; i += blockDim.x) a[i] = __dadd_rn(a[i], a[i + h]);
     __syncthreads();
   }
-  if (threadIdx.x == 0) *mean = __double2float_rn(__ddiv_rn(a[0], static_cast<double>(nb)));
+  // now at most 2*min(size,1024) live values remain: a[0 .. 2h)
+  const int t = threadIdx.x;
+  const int live = static_cast<int>(size < 1024 ? size : 1024);
+  s[t] = t < live ? a[t] : 0.0;
+  __syncthreads();
+  for (int hh = live / 2; hh >= 32; hh /= 2) {
+    if (t < hh) s[t] = __dadd_rn(s[t], s[t + hh]);
+    __syncthreads();
+  }
+  if (t < 32) {
+    double v = s[t];
+    for (int hh = (live < 32 ? live / 2 : 16); hh >= 1; hh /= 2) {
+      const double o = __shfl_down_sync(0xFFFFFFFFu, v, hh);
+      if (t < hh) v = __dadd_rn(v, o);
+    }
+    if (t == 0) *mean = __double2float_rn(__ddiv_rn(v, static_cast<double>(nb)));
+  }
 }
 
 __global__ void __launch_bounds__(256) k_double_quant(const float *__restrict__ absmax, int64_t nb,
