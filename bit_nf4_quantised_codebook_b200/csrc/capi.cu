@@ -77,6 +77,18 @@ SplitPlan choose(int64_t tiles, int64_t k_total, int target_ctas, int min_iters)
   return sp;
 }
 
+// K splits of a skinny product, run as one cluster per output tile: a power of
+// two up to 8 (the portable cluster size), at least two K steps per split.
+SplitPlan choose_cluster(int64_t tiles, int64_t k_total, int target_ctas) {
+  SplitPlan sp;
+  sp.k_iters_total = static_cast<int>(k_total);
+  int s = 1;
+  while (s < 8 && tiles * s * 2 <= target_ctas && k_total >= 4 * s) s *= 2;
+  sp.splits = s;
+  sp.k_iters = static_cast<int>((k_total + s - 1) / s);
+  return sp;
+}
+
 size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 
 int device_sms() {
@@ -141,24 +153,20 @@ LinearPlan make_plan(int op, int64_t M, int64_t N, int64_t K, int r, int num_sms
   }
   pl.rpad = r <= 16 ? 16 : r <= 32 ? 32 : r <= 64 ? 64 : r <= 128 ? 128 : 256;
   const int64_t mt = (M + 127) / 128;
-  pl.sp_t = choose(mt, K / 64, 2 * num_sms, 2);
+  pl.sp_t = choose_cluster(mt, K / 64, 2 * num_sms);
   pl.off_sT = take(static_cast<size_t>(M) * r * 2);
-  pl.off_t_part = take(static_cast<size_t>(pl.sp_t.splits) * M * pl.rpad * 4);
   if (op == QLORA_OP_FORWARD) {
     pl.pair_main = M > 128;
     pl.sp_main = choose((pl.pair_main ? 2 * ((M + 511) / 512) : mt) * ((N + 255) / 256), K / 64, num_sms, 4);
     if (pl.sp_main.splits > 1) pl.off_main_part = take(static_cast<size_t>(pl.sp_main.splits) * M * N * 4);
   } else {
-    pl.sp_u = choose(mt, (N + 63) / 64, 2 * num_sms, 2);
+    pl.sp_u = choose_cluster(mt, (N + 63) / 64, 2 * num_sms);
     pl.pair_dx = M > 128;
     pl.sp_dx = choose((pl.pair_dx ? 2 * ((M + 511) / 512) : mt) * ((K + 255) / 256), (N + 63) / 64, num_sms, 4);
-    pl.sp_da = choose((K + 127) / 128, (M + 63) / 64, 2 * num_sms, 2);
-    pl.sp_db = choose((N + 127) / 128, (M + 63) / 64, 2 * num_sms, 2);
+    pl.sp_da = choose_cluster((K + 127) / 128, (M + 63) / 64, 2 * num_sms);
+    pl.sp_db = choose_cluster((N + 127) / 128, (M + 63) / 64, 2 * num_sms);
     pl.off_sU = take(static_cast<size_t>(M) * r * 2);
-    pl.off_u_part = take(static_cast<size_t>(pl.sp_u.splits) * M * pl.rpad * 4);
     if (pl.sp_dx.splits > 1) pl.off_main_part = take(static_cast<size_t>(pl.sp_dx.splits) * M * K * 4);
-    pl.off_da_part = take(static_cast<size_t>(pl.sp_da.splits) * K * pl.rpad * 4);
-    pl.off_db_part = take(static_cast<size_t>(pl.sp_db.splits) * N * pl.rpad * 4);
   }
   pl.bytes = off;
   return pl;

@@ -24,6 +24,7 @@
 #pragma once
 #include <cstdint>
 #include <cuda.h>
+#include <cuda_bf16.h>
 #include "nf4_decode.cuh"
 #include "ptx.cuh"
 
@@ -31,7 +32,13 @@ namespace qlora {
 
 enum BMode : int { B_TMA_K = 0, B_TMA_MN = 1, B_DQ_K = 2, B_DQ_MN = 3 };
 enum LoraMode : int { LORA_NONE = 0, LORA_B2_MN = 1, LORA_B2_K = 2 };
-enum OutMode : int { OUT_BF16 = 0, OUT_F32 = 1 };
+// OUT_BF16 / OUT_F32: the tile is written as is (OUT_F32 into split partials).
+// OUT_RED_*: the K splits of a tile run as one thread-block cluster (1 x 1 x S);
+// each CTA parks its float32 partial in shared memory and the cluster sums the
+// S partials in rank order through distributed shared memory, scales by
+// p.scale and writes the final tile: bf16 [row][col], float32 [row][col], or
+// float32 transposed [col][row].
+enum OutMode : int { OUT_BF16 = 0, OUT_F32 = 1, OUT_RED_BF16 = 2, OUT_RED_F32 = 3, OUT_RED_F32_T = 4 };
 
 // Bound on the waits that drain in-flight copies and MMAs before exit (independent of
 // the configurable pipeline-wait bound, so a short bound never abandons a copy in flight).
@@ -58,6 +65,10 @@ struct GemmParams {
   unsigned long long timeout_ns;
   uint32_t k_shr16;  // 2^16 (a right shift by 16 done as a high-half multiply)
   uint32_t k_shr1;   // 2^31 (a right shift by 1 likewise)
+  // OUT_RED_* only
+  int cluster;       // K splits = CTAs per cluster along z (1, 2, 4 or 8)
+  int red_cols;      // valid output columns (<= BN)
+  float scale;       // applied to the reduced sum
 };
 
 template <int BN_, int STAGES_, bool A_MN_, int BMODE_, int LORA_, int OUT_>
@@ -80,6 +91,9 @@ struct GemmCfg {
   static constexpr int TMEM_COLS = BN <= 32 ? 32 : BN <= 64 ? 64 : BN <= 128 ? 128 : 256;
   static constexpr int BAR_BYTES = 256;
   static constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + BAR_BYTES + 1024;
+  static constexpr bool RED = OUT >= OUT_RED_BF16;
+  static constexpr int PSTRIDE = BN + 4;  // floats per row of the parked partial (conflict-free rows)
+  static_assert(!RED || 128 * PSTRIDE * 4 <= STAGES * STAGE_BYTES, "partial must fit in the pipeline smem");
   static_assert(BN % 16 == 0 && BN >= 16 && BN <= 256, "UMMA N");
   static_assert(!DQ || BN == 256, "dequant tiles are 256 wide");
   static_assert(STAGE_BYTES % 1024 == 0, "swizzle atoms need 1 KiB alignment");
@@ -269,7 +283,35 @@ __global__ void __launch_bounds__(C::NUM_THREADS, 1)
       }
     }
     // ------------------------------------------------------------ epilogue (warps 2..5)
-    if (warp < 6) {
+    if (C::RED && warp < 6) {
+      // park this CTA's float32 partial (row = TMEM lane) in shared memory
+      bool ok = true;
+      if (lane == 0) ok = mbar_wait_bounded(acc_full, 0, abort_flag, p.dev_err, p.timeout_ns);
+      ok = __shfl_sync(0xFFFFFFFFu, ok ? 1 : 0, 0) != 0;
+      if (ok && !*abort_flag) {
+        __syncwarp();
+        tc_fence_after();
+        const int q = warp & 3;
+        const int row = q * 32 + lane;
+        float *prow = reinterpret_cast<float *>(smem) + row * C::PSTRIDE;
+        for (int c0 = 0; c0 < C::BN; c0 += 32) {
+          uint32_t v[32];
+          tmem_ld32(tmem_acc + (static_cast<uint32_t>(q * 32) << 16) + c0, v);
+          tmem_ld_wait();
+          const int ncol = C::BN - c0 < 32 ? C::BN - c0 : 32;
+#pragma unroll
+          for (int g = 0; g < 8; ++g) {
+            if (4 * g < ncol) {
+              float4 f = n_total > 0 ? make_float4(__uint_as_float(v[4 * g]), __uint_as_float(v[4 * g + 1]),
+                                                   __uint_as_float(v[4 * g + 2]), __uint_as_float(v[4 * g + 3]))
+                                     : make_float4(0.f, 0.f, 0.f, 0.f);
+              *reinterpret_cast<float4 *>(prow + c0 + 4 * g) = f;
+            }
+          }
+        }
+      }
+    }
+    if (!C::RED && warp < 6) {
       bool ok = true;
       if (lane == 0) ok = mbar_wait_bounded(acc_full, 0, abort_flag, p.dev_err, p.timeout_ns);
       ok = __shfl_sync(0xFFFFFFFFu, ok ? 1 : 0, 0) != 0;
@@ -312,6 +354,65 @@ __global__ void __launch_bounds__(C::NUM_THREADS, 1)
         }
       }
     }
+  }
+
+  if (C::RED) {
+    // ------------------------------------------------------------ in-cluster split reduction
+    cluster_sync();  // every CTA's partial is parked
+    const int S = p.cluster;
+    const int j = static_cast<int>(cluster_ctarank());
+    const int R = 128 / S;  // rows this CTA finishes
+    const uint32_t pbase = smem_base + static_cast<uint32_t>(j * R) * C::PSTRIDE * 4;
+    const int ncol4 = (p.red_cols + 3) / 4;  // red_cols is a multiple of 8
+    const int nval = R * ncol4;
+    for (int v = threadIdx.x; v < nval; v += C::NUM_THREADS) {
+      int row, c4;
+      if (C::OUT == OUT_RED_F32_T) {  // consecutive threads -> consecutive rows (coalesced transposed writes)
+        row = v % R;
+        c4 = v / R;
+      } else {  // consecutive threads -> consecutive columns
+        row = v / ncol4;
+        c4 = v % ncol4;
+      }
+      const uint32_t off = pbase + static_cast<uint32_t>(row * C::PSTRIDE + 4 * c4) * 4;
+      float4 part[8];
+#pragma unroll
+      for (int qr = 0; qr < 8; ++qr)
+        if (qr < S) part[qr] = ld_shared_cluster_v4(mapa_shared(off, static_cast<uint32_t>(qr)));
+      float4 acc = part[0];
+#pragma unroll
+      for (int qr = 1; qr < 8; ++qr) {
+        if (qr < S) {
+          acc.x += part[qr].x;
+          acc.y += part[qr].y;
+          acc.z += part[qr].z;
+          acc.w += part[qr].w;
+        }
+      }
+      acc.x *= p.scale;
+      acc.y *= p.scale;
+      acc.z *= p.scale;
+      acc.w *= p.scale;
+      const int grow = m0 + j * R + row;
+      const int col = 4 * c4;
+      if (grow < p.rows) {
+        if (C::OUT == OUT_RED_BF16) {
+          uint2 pk;
+          pk.x = pack_bf16x2(acc.x, acc.y);
+          pk.y = pack_bf16x2(acc.z, acc.w);
+          *reinterpret_cast<uint2 *>(reinterpret_cast<uint16_t *>(p.out) + static_cast<int64_t>(grow) * p.ld_out + col) = pk;
+        } else if (C::OUT == OUT_RED_F32) {
+          *reinterpret_cast<float4 *>(reinterpret_cast<float *>(p.out) + static_cast<int64_t>(grow) * p.ld_out + col) = acc;
+        } else {
+          float *o = reinterpret_cast<float *>(p.out);
+          o[static_cast<int64_t>(col + 0) * p.ld_out + grow] = acc.x;
+          o[static_cast<int64_t>(col + 1) * p.ld_out + grow] = acc.y;
+          o[static_cast<int64_t>(col + 2) * p.ld_out + grow] = acc.z;
+          o[static_cast<int64_t>(col + 3) * p.ld_out + grow] = acc.w;
+        }
+      }
+    }
+    cluster_sync();  // no CTA leaves while a peer may still read its partial
   }
 
   tc_fence_before();

@@ -11,7 +11,8 @@
 // never in HBM), with the LoRA product appended as extra K steps into the same
 // TMEM accumulator.  The four skinny products (output width r) run in the same
 // GEMM template with both operands streamed by TMA and the long reduction split
-// across CTAs; partial sums are reduced in a fixed order by finalize kernels.
+// across the CTAs of a thread-block cluster, summed in rank order through
+// distributed shared memory (no partial buffers, no extra launch).
 #include <algorithm>
 #include <cstdint>
 #include <cstring>
@@ -29,13 +30,15 @@ using CfgFwd = GemmCfg<256, 4, false, B_DQ_K, LORA_B2_MN, OUT_BF16>;
 using CfgFwdSplit = GemmCfg<256, 4, false, B_DQ_K, LORA_B2_MN, OUT_F32>;
 using CfgBwd = GemmCfg<256, 4, false, B_DQ_MN, LORA_B2_K, OUT_BF16>;
 using CfgBwdSplit = GemmCfg<256, 4, false, B_DQ_MN, LORA_B2_K, OUT_F32>;
-// skinny: output width r_pad (16..256); instantiated for the r buckets below
+// skinny: output width r_pad (16..256); K splits reduced inside a cluster
 template <int BN>
-using CfgT = GemmCfg<BN, 4, false, B_TMA_MN, LORA_NONE, OUT_F32>;  // X·A        (A-op X K-major, B-op Aᵀ MN-major)
+using CfgT = GemmCfg<BN, 4, false, B_TMA_MN, LORA_NONE, OUT_RED_BF16>;  // s·X·A   (X K-major, Aᵀ MN-major)
 template <int BN>
-using CfgU = GemmCfg<BN, 4, false, B_TMA_K, LORA_NONE, OUT_F32>;   // dY·Bᵀ      (B-op B K-major)
+using CfgU = GemmCfg<BN, 4, false, B_TMA_K, LORA_NONE, OUT_RED_BF16>;   // s·dY·Bᵀ (B K-major)
 template <int BN>
-using CfgW = GemmCfg<BN, 4, true, B_TMA_MN, LORA_NONE, OUT_F32>;   // Xᵀ·sU, dYᵀ·sT (both MN-major)
+using CfgDA = GemmCfg<BN, 4, true, B_TMA_MN, LORA_NONE, OUT_RED_F32>;   // Xᵀ·sU   (both MN-major)
+template <int BN>
+using CfgDB = GemmCfg<BN, 4, true, B_TMA_MN, LORA_NONE, OUT_RED_F32_T>; // (dYᵀ·sT)ᵀ written as dB
 
 template <class C>
 static cudaError_t prepare() {
@@ -52,6 +55,29 @@ static cudaError_t launch(dim3 grid, const TmaMaps &m, const GemmParams &p, cuda
   if (e != cudaSuccess) return e;
   gemm_kernel<C><<<grid, C::NUM_THREADS, C::SMEM_BYTES, st>>>(m.a, m.b, m.a2, m.b2, p);
   count_launches(1);
+  return cudaGetLastError();
+}
+
+// Launch with clusters of 1 x 1 x cz CTAs (the K splits of one output tile).
+template <class C>
+static cudaError_t launch_cluster(dim3 grid, int cz, const TmaMaps &m, const GemmParams &p, cudaStream_t st) {
+  cudaError_t e = prepare<C>();
+  if (e != cudaSuccess) return e;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = dim3(C::NUM_THREADS, 1, 1);
+  cfg.dynamicSmemBytes = C::SMEM_BYTES;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 1;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = static_cast<unsigned>(cz);
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  e = cudaLaunchKernelEx(&cfg, gemm_kernel<C>, m.a, m.b, m.a2, m.b2, p);
+  count_launches(1);
+  if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }
 
@@ -98,52 +124,6 @@ __global__ void k_finalize_bf16(const float *__restrict__ part, int splits, int6
   *reinterpret_cast<uint2 *>(out + row * ldo + c) = pk;
 }
 
-__global__ void k_finalize_f32(const float *__restrict__ part, int splits, int64_t split_stride, int64_t rows,
-                               int cols, int ldp, float scale, float *__restrict__ out, int64_t ldo) {
-  const int64_t idx = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
-  const int64_t nvec = rows * (cols / 4);
-  if (idx >= nvec) return;
-  const int64_t row = idx / (cols / 4);
-  const int c = static_cast<int>(idx % (cols / 4)) * 4;
-  float4 acc = *reinterpret_cast<const float4 *>(part + row * ldp + c);
-  for (int s = 1; s < splits; ++s) {
-    const float4 v = *reinterpret_cast<const float4 *>(part + s * split_stride + row * ldp + c);
-    acc.x += v.x;
-    acc.y += v.y;
-    acc.z += v.z;
-    acc.w += v.w;
-  }
-  acc.x *= scale;
-  acc.y *= scale;
-  acc.z *= scale;
-  acc.w *= scale;
-  *reinterpret_cast<float4 *>(out + row * ldo + c) = acc;
-}
-
-// out[c, row] = scale * sum_s part[s][row][c]   (transposing finalize, 32x32 tiles)
-__global__ void k_finalize_f32_t(const float *__restrict__ part, int splits, int64_t split_stride, int64_t rows,
-                                 int cols, int ldp, float scale, float *__restrict__ out, int64_t ldo) {
-  __shared__ float tile[32][33];
-  const int64_t r0 = static_cast<int64_t>(blockIdx.x) * 32;
-  const int c0 = blockIdx.y * 32;
-  for (int i = threadIdx.y; i < 32; i += blockDim.y) {
-    const int64_t row = r0 + i;
-    const int c = c0 + threadIdx.x;
-    float acc = 0.f;
-    if (row < rows && c < cols) {
-      acc = part[row * ldp + c];
-      for (int s = 1; s < splits; ++s) acc += part[s * split_stride + row * ldp + c];
-    }
-    tile[i][threadIdx.x] = acc * scale;
-  }
-  __syncthreads();
-  for (int i = threadIdx.y; i < 32; i += blockDim.y) {
-    const int c = c0 + i;
-    const int64_t row = r0 + threadIdx.x;
-    if (row < rows && c < cols) out[static_cast<int64_t>(c) * ldo + row] = tile[threadIdx.x][i];
-  }
-}
-
 static cudaError_t finalize_bf16(const float *part, int splits, int64_t split_stride, int64_t rows, int cols,
                                  int ldp, float scale, uint16_t *out, int64_t ldo, cudaStream_t st) {
   const int64_t n = rows * (cols / 4);
@@ -153,44 +133,19 @@ static cudaError_t finalize_bf16(const float *part, int splits, int64_t split_st
   count_launches(1);
   return cudaGetLastError();
 }
-static cudaError_t finalize_f32(const float *part, int splits, int64_t split_stride, int64_t rows, int cols, int ldp,
-                                float scale, float *out, int64_t ldo, cudaStream_t st) {
-  const int64_t n = rows * (cols / 4);
-  const int64_t grid = (n + 255) / 256;
-  k_finalize_f32<<<static_cast<unsigned>(grid), 256, 0, st>>>(part, splits, split_stride, rows, cols, ldp, scale, out,
-                                                                ldo);
-  count_launches(1);
-  return cudaGetLastError();
-}
-static cudaError_t finalize_f32_t(const float *part, int splits, int64_t split_stride, int64_t rows, int cols,
-                                  int ldp, float scale, float *out, int64_t ldo, cudaStream_t st) {
-  dim3 grid(static_cast<unsigned>((rows + 31) / 32), static_cast<unsigned>((cols + 31) / 32));
-  k_finalize_f32_t<<<grid, dim3(32, 8), 0, st>>>(part, splits, split_stride, rows, cols, ldp, scale, out, ldo);
-  count_launches(1);
-  return cudaGetLastError();
-}
-
 // ---------------------------------------------------------------- skinny GEMM dispatch over r buckets
-enum SkinnyKind { SK_T = 0, SK_U = 1, SK_W = 2 };
+enum SkinnyKind { SK_T = 0, SK_U = 1, SK_DA = 2, SK_DB = 3 };
 
 template <template <int> class CF>
-static cudaError_t launch_bucket(int rpad, dim3 grid, const TmaMaps &m, const GemmParams &p, cudaStream_t st) {
-  switch (rpad) {
-    case 16: return launch<CF<16>>(grid, m, p, st);
-    case 32: return launch<CF<32>>(grid, m, p, st);
-    case 64: return launch<CF<64>>(grid, m, p, st);
-    case 128: return launch<CF<128>>(grid, m, p, st);
-    case 256: return launch<CF<256>>(grid, m, p, st);
-    default: return cudaErrorInvalidValue;
-  }
-}
-
-static cudaError_t launch_skinny(SkinnyKind kind, int rpad, dim3 grid, const TmaMaps &m, const GemmParams &p,
+static cudaError_t launch_bucket(int rpad, dim3 grid, int cz, const TmaMaps &m, const GemmParams &p,
                                  cudaStream_t st) {
-  switch (kind) {
-    case SK_T: return launch_bucket<CfgT>(rpad, grid, m, p, st);
-    case SK_U: return launch_bucket<CfgU>(rpad, grid, m, p, st);
-    default: return launch_bucket<CfgW>(rpad, grid, m, p, st);
+  switch (rpad) {
+    case 16: return launch_cluster<CF<16>>(grid, cz, m, p, st);
+    case 32: return launch_cluster<CF<32>>(grid, cz, m, p, st);
+    case 64: return launch_cluster<CF<64>>(grid, cz, m, p, st);
+    case 128: return launch_cluster<CF<128>>(grid, cz, m, p, st);
+    case 256: return launch_cluster<CF<256>>(grid, cz, m, p, st);
+    default: return cudaErrorInvalidValue;
   }
 }
 
@@ -202,23 +157,33 @@ static GemmParams base_params(const LaunchCtx &c) {
   p.lv = c.levels;
   p.k_shr16 = 1u << 16;
   p.k_shr1 = 1u << 31;
+  p.cluster = 1;
+  p.scale = 1.0f;
   return p;
 }
 
-// Skinny product: D[rows x rpad] = sum over `red` (split) of Aop·Bopᵀ, written as
-// float32 partials [splits][rows][rpad] into `part`.
-static cudaError_t run_skinny(SkinnyKind kind, const LaunchCtx &c, const SplitPlan &sp, int rpad, int rows,
-                              const TmaMaps &maps, float *part) {
+// Skinny product: D[rows x r] = scale · sum over the reduction of Aop·Bopᵀ, the
+// reduction split over the sp.splits CTAs of one cluster and summed in-cluster.
+// Writes out[row][c] (ld_out) or, for SK_DB, out[c][row].
+static cudaError_t run_skinny(SkinnyKind kind, const LaunchCtx &c, const SplitPlan &sp, int rpad, int r, int rows,
+                              float scale, const TmaMaps &maps, void *out, int64_t ld_out) {
   GemmParams p = base_params(c);
   p.rows = rows;
   p.cols = rpad;
   p.k_iters = sp.k_iters;
   p.k_iters_total = sp.k_iters_total;
-  p.out = part;
-  p.ld_out = rpad;
-  p.split_stride = static_cast<int64_t>(rows) * rpad;
+  p.out = out;
+  p.ld_out = ld_out;
+  p.cluster = sp.splits;
+  p.red_cols = r;
+  p.scale = scale;
   dim3 grid(static_cast<unsigned>((rows + 127) / 128), 1, static_cast<unsigned>(sp.splits));
-  return launch_skinny(kind, rpad, grid, maps, p, c.stream);
+  switch (kind) {
+    case SK_T: return launch_bucket<CfgT>(rpad, grid, sp.splits, maps, p, c.stream);
+    case SK_U: return launch_bucket<CfgU>(rpad, grid, sp.splits, maps, p, c.stream);
+    case SK_DA: return launch_bucket<CfgDA>(rpad, grid, sp.splits, maps, p, c.stream);
+    default: return launch_bucket<CfgDB>(rpad, grid, sp.splits, maps, p, c.stream);
+  }
 }
 
 // ---------------------------------------------------------------- fused dequant GEMM
@@ -276,32 +241,27 @@ static cudaError_t run_fused(bool fwd, const LaunchCtx &c, const qlora_nf4_weigh
 }
 
 // ---------------------------------------------------------------- forward
+// sT = bf16(s·X·A)  (A-op X [M,K] K-major; B-op Aᵀ: A [K,r] read MN-major)
+static cudaError_t run_t(const LaunchCtx &c, const uint16_t *X, int64_t M, int K, const uint16_t *A, int r, float s,
+                         uint16_t *sT, const LinearPlan &pl) {
+  TmaMaps m;
+  if (!map_bf16_kmajor(&m.a, X, K, M, 128) || !map_bf16_mn(&m.b, A, r, K)) return cudaErrorInvalidValue;
+  m.a2 = m.a;
+  m.b2 = m.b;
+  return run_skinny(SK_T, c, pl.sp_t, pl.rpad, r, static_cast<int>(M), s, m, sT, r);
+}
+
 cudaError_t run_forward(const LaunchCtx &c, const qlora_nf4_weight &w, const uint16_t *X, int64_t M,
                         const uint16_t *A, const uint16_t *B, int r, float s, uint16_t *Y, uint16_t *T_save,
                         const LinearPlan &pl, uint8_t *ws) {
   cudaError_t e;
-  const int N = static_cast<int>(w.N), K = static_cast<int>(w.K);
-  float *t_part = reinterpret_cast<float *>(ws + pl.off_t_part);
+  const int K = static_cast<int>(w.K);
   uint16_t *sT = T_save ? T_save : reinterpret_cast<uint16_t *>(ws + pl.off_sT);
-  // T = X·A  (A-op X [M,K] K-major; B-op Aᵀ: A [K,r] read MN-major)
-  {
-    TmaMaps m;
-    if (!map_bf16_kmajor(&m.a, X, K, M, 128) || !map_bf16_mn(&m.b, A, r, K)) return cudaErrorInvalidValue;
-    m.a2 = m.a;
-    m.b2 = m.b;
-    if ((e = run_skinny(SK_T, c, pl.sp_t, pl.rpad, static_cast<int>(M), m, t_part)) != cudaSuccess) return e;
-    if ((e = finalize_bf16(t_part, pl.sp_t.splits, M * pl.rpad, M, r, pl.rpad, s, sT, r, c.stream)) != cudaSuccess)
-      return e;
-  }
+  if ((e = run_t(c, X, M, K, A, r, s, sT, pl)) != cudaSuccess) return e;
   // Y = X·W_hatᵀ + sT·B
-  {
-    const TimingHooks &hk = timing_hooks();
-    float *part = reinterpret_cast<float *>(ws + pl.off_main_part);
-    if ((e = run_fused(true, c, w, X, M, sT, B, r, Y, pl.pair_main, pl.sp_main, part, hk.fwd_begin, hk.fwd_end)) !=
-        cudaSuccess)
-      return e;
-  }
-  return cudaSuccess;
+  const TimingHooks &hk = timing_hooks();
+  float *part = reinterpret_cast<float *>(ws + pl.off_main_part);
+  return run_fused(true, c, w, X, M, sT, B, r, Y, pl.pair_main, pl.sp_main, part, hk.fwd_begin, hk.fwd_end);
 }
 
 // ---------------------------------------------------------------- backward
@@ -313,29 +273,18 @@ cudaError_t run_backward(const LaunchCtx &c, const qlora_nf4_weight &w, const ui
   const uint16_t *sT = T_saved;
   if (!sT) {  // recompute bf16(s·X·A)
     uint16_t *sT_ws = reinterpret_cast<uint16_t *>(ws + pl.off_sT);
-    float *t_part = reinterpret_cast<float *>(ws + pl.off_t_part);
-    TmaMaps m;
-    if (!map_bf16_kmajor(&m.a, X, K, M, 128) || !map_bf16_mn(&m.b, A, r, K)) return cudaErrorInvalidValue;
-    m.a2 = m.a;
-    m.b2 = m.b;
-    if ((e = run_skinny(SK_T, c, pl.sp_t, pl.rpad, static_cast<int>(M), m, t_part)) != cudaSuccess) return e;
-    if ((e = finalize_bf16(t_part, pl.sp_t.splits, M * pl.rpad, M, r, pl.rpad, s, sT_ws, r, c.stream)) !=
-        cudaSuccess)
-      return e;
+    if ((e = run_t(c, X, M, K, A, r, s, sT_ws, pl)) != cudaSuccess) return e;
     sT = sT_ws;
   }
   uint16_t *sU = reinterpret_cast<uint16_t *>(ws + pl.off_sU);
-  // U = dY·Bᵀ  (A-op dY [M,N] K-major; B-op B [r,N] K-major)
+  // sU = bf16(s·dY·Bᵀ)  (A-op dY [M,N] K-major; B-op B [r,N] K-major)
   {
-    float *u_part = reinterpret_cast<float *>(ws + pl.off_u_part);
     TmaMaps m;
     if (!map_bf16_kmajor(&m.a, dY, N, M, 128) || !map_bf16_kmajor(&m.b, B, N, r, pl.rpad))
       return cudaErrorInvalidValue;
     m.a2 = m.a;
     m.b2 = m.b;
-    if ((e = run_skinny(SK_U, c, pl.sp_u, pl.rpad, static_cast<int>(M), m, u_part)) != cudaSuccess) return e;
-    if ((e = finalize_bf16(u_part, pl.sp_u.splits, M * pl.rpad, M, r, pl.rpad, s, sU, r, c.stream)) != cudaSuccess)
-      return e;
+    if ((e = run_skinny(SK_U, c, pl.sp_u, pl.rpad, r, static_cast<int>(M), s, m, sU, r)) != cudaSuccess) return e;
   }
   // dX = dY·W_hat + sU·Aᵀ
   if (dX) {
@@ -347,27 +296,19 @@ cudaError_t run_backward(const LaunchCtx &c, const qlora_nf4_weight &w, const ui
   }
   // dA = Xᵀ·sU : D[K x r] (A-op Xᵀ: X [M,K] MN-major; B-op sUᵀ: sU [M,r] MN-major)
   {
-    float *part = reinterpret_cast<float *>(ws + pl.off_da_part);
     TmaMaps m;
     if (!map_bf16_mn(&m.a, X, K, M) || !map_bf16_mn(&m.b, sU, r, M)) return cudaErrorInvalidValue;
     m.a2 = m.a;
     m.b2 = m.b;
-    if ((e = run_skinny(SK_W, c, pl.sp_da, pl.rpad, K, m, part)) != cudaSuccess) return e;
-    if ((e = finalize_f32(part, pl.sp_da.splits, static_cast<int64_t>(K) * pl.rpad, K, r, pl.rpad, 1.0f, dA, r,
-                          c.stream)) != cudaSuccess)
-      return e;
+    if ((e = run_skinny(SK_DA, c, pl.sp_da, pl.rpad, r, K, 1.0f, m, dA, r)) != cudaSuccess) return e;
   }
-  // dB = sTᵀ·dY : computed as D[N x r] = dYᵀ·sT, then transposed by the finalize
+  // dB = sTᵀ·dY : D[N x r] = dYᵀ·sT, written transposed into dB [r, N]
   {
-    float *part = reinterpret_cast<float *>(ws + pl.off_db_part);
     TmaMaps m;
     if (!map_bf16_mn(&m.a, dY, N, M) || !map_bf16_mn(&m.b, sT, r, M)) return cudaErrorInvalidValue;
     m.a2 = m.a;
     m.b2 = m.b;
-    if ((e = run_skinny(SK_W, c, pl.sp_db, pl.rpad, N, m, part)) != cudaSuccess) return e;
-    if ((e = finalize_f32_t(part, pl.sp_db.splits, static_cast<int64_t>(N) * pl.rpad, N, r, pl.rpad, 1.0f, dB, N,
-                            c.stream)) != cudaSuccess)
-      return e;
+    if ((e = run_skinny(SK_DB, c, pl.sp_db, pl.rpad, r, N, 1.0f, m, dB, N)) != cudaSuccess) return e;
   }
   return cudaSuccess;
 }

@@ -31,8 +31,7 @@ struct LinearPlan {
   int rpad = 16;
   SplitPlan sp_t, sp_u, sp_main, sp_dx, sp_da, sp_db;
   bool pair_main = false, pair_dx = false;  // CTA-pair kernel for the fused GEMMs
-  size_t off_sT = 0, off_t_part = 0, off_sU = 0, off_u_part = 0, off_main_part = 0, off_da_part = 0,
-         off_db_part = 0;
+  size_t off_sT = 0, off_sU = 0, off_main_part = 0;
   size_t off_absmax = 0, off_gsum = 0;
   int64_t gsum_size = 0;
   size_t bytes = 0;
