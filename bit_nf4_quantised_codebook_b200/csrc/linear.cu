@@ -21,6 +21,7 @@
 #include "gemm.cuh"
 #include "gemm_pair.cuh"
 #include "internal.h"
+#include "launch.cuh"
 #include "linear_plan.h"
 
 namespace qlora {
@@ -53,9 +54,7 @@ template <class C>
 static cudaError_t launch(dim3 grid, const TmaMaps &m, const GemmParams &p, cudaStream_t st) {
   cudaError_t e = prepare<C>();
   if (e != cudaSuccess) return e;
-  gemm_kernel<C><<<grid, C::NUM_THREADS, C::SMEM_BYTES, st>>>(m.a, m.b, m.a2, m.b2, p);
-  count_launches(1);
-  return cudaGetLastError();
+  return launch_k(gemm_kernel<C>, grid, dim3(C::NUM_THREADS), C::SMEM_BYTES, st, 1, m.a, m.b, m.a2, m.b2, p);
 }
 
 // Launch with clusters of 1 x 1 x cz CTAs (the K splits of one output tile).
@@ -63,22 +62,8 @@ template <class C>
 static cudaError_t launch_cluster(dim3 grid, int cz, const TmaMaps &m, const GemmParams &p, cudaStream_t st) {
   cudaError_t e = prepare<C>();
   if (e != cudaSuccess) return e;
-  cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = grid;
-  cfg.blockDim = dim3(C::NUM_THREADS, 1, 1);
-  cfg.dynamicSmemBytes = C::SMEM_BYTES;
-  cfg.stream = st;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeClusterDimension;
-  attr[0].val.clusterDim.x = 1;
-  attr[0].val.clusterDim.y = 1;
-  attr[0].val.clusterDim.z = static_cast<unsigned>(cz);
-  cfg.attrs = attr;
-  cfg.numAttrs = 1;
-  e = cudaLaunchKernelEx(&cfg, gemm_kernel<C>, m.a, m.b, m.a2, m.b2, p);
-  count_launches(1);
-  if (e != cudaSuccess) return e;
-  return cudaGetLastError();
+  return launch_k(gemm_kernel<C>, grid, dim3(C::NUM_THREADS), C::SMEM_BYTES, st, static_cast<unsigned>(cz), m.a,
+                  m.b, m.a2, m.b2, p);
 }
 
 using PairFwd = PairCfg<4, B_DQ_K, LORA_B2_MN, OUT_BF16, 2>;
@@ -96,15 +81,15 @@ static cudaError_t launch_pair(dim3 grid, const TmaMaps &m, const GemmParams &p,
     if (e != cudaSuccess) return e;
     prepared = true;
   }
-  gemm_pair_kernel<C><<<grid, C::NUM_THREADS, C::SMEM_BYTES, st>>>(m.a, m.b, m.a2, m.b2, p);
-  count_launches(1);
-  return cudaGetLastError();
+  return launch_k(gemm_pair_kernel<C>, grid, dim3(C::NUM_THREADS), C::SMEM_BYTES, st, 1, m.a, m.b, m.a2, m.b2, p);
 }
 
 // ---------------------------------------------------------------- finalize kernels
 // out[row, c] = cvt(scale * sum_s part[s][row][c]), c < cols, sequential over s.
 __global__ void k_finalize_bf16(const float *__restrict__ part, int splits, int64_t split_stride, int64_t rows,
                                 int cols, int ldp, float scale, uint16_t *__restrict__ out, int64_t ldo) {
+  pdl_launch_dependents();
+  pdl_wait();
   const int64_t idx = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
   const int64_t nvec = rows * (cols / 4);
   if (idx >= nvec) return;
@@ -128,10 +113,8 @@ static cudaError_t finalize_bf16(const float *part, int splits, int64_t split_st
                                  int ldp, float scale, uint16_t *out, int64_t ldo, cudaStream_t st) {
   const int64_t n = rows * (cols / 4);
   const int64_t grid = (n + 255) / 256;
-  k_finalize_bf16<<<static_cast<unsigned>(grid), 256, 0, st>>>(part, splits, split_stride, rows, cols, ldp, scale,
-                                                                 out, ldo);
-  count_launches(1);
-  return cudaGetLastError();
+  return launch_k(k_finalize_bf16, dim3(static_cast<unsigned>(grid)), dim3(256), 0, st, 1,
+                  static_cast<const float *>(part), splits, split_stride, rows, cols, ldp, scale, out, ldo);
 }
 // ---------------------------------------------------------------- skinny GEMM dispatch over r buckets
 enum SkinnyKind { SK_T = 0, SK_U = 1, SK_DA = 2, SK_DB = 3 };

@@ -21,6 +21,7 @@
 #include "internal.h"
 #include "nf4_decode.cuh"
 #include "nf4_quant.cuh"
+#include "launch.cuh"
 
 namespace qlora {
 
@@ -56,10 +57,12 @@ __global__ void __launch_bounds__(256, 2) k_quant_blocks(const uint16_t *__restr
                                                        int *dev_err) {
   __shared__ float s_amax[256];
   __shared__ CodeBucket s_tab[kBuckets];
+  pdl_launch_dependents();
   if (threadIdx.x < kBuckets) s_tab[threadIdx.x] = make_bucket(threadIdx.x, thr.t);
   const int64_t g = blockIdx.x;
   const int part = threadIdx.x & 7;  // 8-element chunk of the block
   const int sub = threadIdx.x >> 3;  // block within the pass
+  pdl_wait();
   // all eight 16-byte loads of this thread in flight at once
   uint4 raw[8];
 #pragma unroll
@@ -133,6 +136,8 @@ __global__ void __launch_bounds__(256, 2) k_quant_blocks(const uint16_t *__restr
 __global__ void __launch_bounds__(1024) k_mean_tree(double *__restrict__ a, int64_t ng, int64_t size, int64_t nb,
                                                      float *__restrict__ mean) {
   __shared__ double s[1024];
+  pdl_launch_dependents();
+  pdl_wait();
   for (int64_t i = ng + threadIdx.x; i < size; i += blockDim.x) a[i] = 0.0;
   __syncthreads();
   int64_t h = size / 2;
@@ -163,6 +168,8 @@ __global__ void __launch_bounds__(256) k_double_quant(const float *__restrict__ 
                                                        const float *__restrict__ mean, uint8_t *__restrict__ c2q,
                                                        float *__restrict__ c1) {
   __shared__ float s_red[8];
+  pdl_launch_dependents();
+  pdl_wait();
   const int64_t g = blockIdx.x;
   const int64_t b = g * 256 + threadIdx.x;
   const bool valid = b < nb;
@@ -186,6 +193,8 @@ __global__ void __launch_bounds__(256) k_double_quant(const float *__restrict__ 
 __global__ void __launch_bounds__(256) k_dequant(const uint8_t *__restrict__ codes, const uint8_t *__restrict__ c2q,
                                                   const float *__restrict__ c1, const float *__restrict__ mean,
                                                   int64_t nb, Nf4Levels lv, uint16_t *__restrict__ out) {
+  pdl_launch_dependents();
+  pdl_wait();
   const int64_t b = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
   if (b >= nb) return;
   const float c2h = reconstruct_c2(c2q[b], c1[b >> 8], *mean);
@@ -207,19 +216,20 @@ cudaError_t launch_quantize(const uint16_t *W, int64_t nb, uint8_t *codes, uint8
                             float *ws_absmax, double *ws_gsum, int64_t gsum_size, const Nf4Thresholds &thr,
                             int *dev_err, cudaStream_t st) {
   const int64_t ng = (nb + 255) / 256;
-  k_quant_blocks<<<static_cast<unsigned>(ng), 256, 0, st>>>(W, nb, codes, ws_absmax, ws_gsum, thr, dev_err);
-  k_mean_tree<<<1, 1024, 0, st>>>(ws_gsum, ng, gsum_size, nb, mean);
-  k_double_quant<<<static_cast<unsigned>(ng), 256, 0, st>>>(ws_absmax, nb, mean, c2q, c1);
-  count_launches(3);
-  return cudaGetLastError();
+  cudaError_t e = launch_k(k_quant_blocks, dim3(static_cast<unsigned>(ng)), dim3(256), 0, st, 1, W, nb, codes,
+                           ws_absmax, ws_gsum, thr, dev_err);
+  if (e != cudaSuccess) return e;
+  e = launch_k(k_mean_tree, dim3(1), dim3(1024), 0, st, 1, ws_gsum, ng, gsum_size, nb, mean);
+  if (e != cudaSuccess) return e;
+  return launch_k(k_double_quant, dim3(static_cast<unsigned>(ng)), dim3(256), 0, st, 1,
+                  static_cast<const float *>(ws_absmax), nb, static_cast<const float *>(mean), c2q, c1);
 }
 
 cudaError_t launch_dequantize(const uint8_t *codes, const uint8_t *c2q, const float *c1, const float *mean,
                               int64_t nb, const Nf4Levels &lv, uint16_t *out, cudaStream_t st) {
   const int64_t grid = (nb + 255) / 256;
-  k_dequant<<<static_cast<unsigned>(grid), 256, 0, st>>>(codes, c2q, c1, mean, nb, lv, out);
-  count_launches(1);
-  return cudaGetLastError();
+  return launch_k(k_dequant, dim3(static_cast<unsigned>(grid)), dim3(256), 0, st, 1, codes, c2q, c1, mean, nb, lv,
+                  out);
 }
 
 }  // namespace qlora
