@@ -22,8 +22,8 @@ DESIGN.md):
   * the 8-bit float of the second quantisation is OCP FP8 E4M3FN, rounded to
     nearest-even and saturated at +-448 ([P2] "an 8-bit float", [P5] "FP8");
   * the mean subtracted before the second quantisation is one float32 value
-    per tensor, summed in a fixed order (per-group sequential float64 sums,
-    then a power-of-two pairwise tree);
+    per tensor, summed in a fixed order (a float64 pairwise tree within each
+    group of 256 blocks, then a pairwise tree over the group sums);
   * a group is 256 consecutive blocks of the flat block index; the last group
     may be partial.
 """
@@ -194,30 +194,36 @@ def unpack_nibbles(packed: np.ndarray) -> np.ndarray:
 # ---------------------------------------------------------------------------
 # double quantisation ([P2] §Double quantization; [P5])
 # ---------------------------------------------------------------------------
+def _pairwise_tree(a: np.ndarray) -> np.ndarray:
+    """Pairwise tree along the last axis (length a power of two): for
+    h = n/2, n/4, ..., 1 every a[i] (i < h) becomes a[i] + a[i+h]."""
+    a = a.copy()
+    h = a.shape[-1] // 2
+    while h >= 1:
+        a[..., :h] = a[..., :h] + a[..., h:2 * h]
+        h //= 2
+    return a[..., 0]
+
+
 def fixed_order_mean(c2: np.ndarray) -> np.float32:
-    """Mean of the block constants in a fixed summation order: per group of
-    256 blocks a sequential float64 sum, then the group sums padded with zeros
-    to a power of two and added pairwise (a[i] += a[i+h], h halving), finally
-    one float64 division by the block count rounded to float32."""
+    """Mean of the block constants in one fixed float64 summation order: a
+    pairwise tree over each group of 256 blocks (the last group zero-padded),
+    then the same kind of tree over the group sums (zero-padded to a power of
+    two), then one float64 division by the block count rounded to float32.
+    (The pages only say the mean is subtracted first; the order is this
+    library's reading, chosen so the sum is deterministic and parallel.)"""
     c = np.asarray(c2, _F32).astype(_F64)
     nb = c.size
     ng = -(-nb // GROUP)
     padded = np.zeros(ng * GROUP, _F64)
     padded[:nb] = c
-    tab = padded.reshape(ng, GROUP)
-    acc = np.zeros(ng, _F64)
-    for j in range(GROUP):                    # sequential within a group
-        acc = acc + tab[:, j]
+    group_sums = _pairwise_tree(padded.reshape(ng, GROUP))
     size = 1
     while size < ng:
         size *= 2
     a = np.zeros(size, _F64)
-    a[:ng] = acc
-    h = size // 2
-    while h >= 1:
-        a[:h] = a[:h] + a[h:2 * h]
-        h //= 2
-    return _F32(a[0] / nb)
+    a[:ng] = group_sums
+    return _F32(_pairwise_tree(a) / nb)
 
 
 def double_quantize(c2: np.ndarray) -> tuple[np.ndarray, np.ndarray, np.float32]:

@@ -138,13 +138,17 @@ def test_fixed_order_mean_vs_exact_sum():
 
 
 def test_fixed_order_mean_is_order_defined():
-    # a sum whose float64 value depends on order: the defined order gives this exact result
-    c = np.array([1.0, 2.0 ** -30] * 128 + [1.0] * 128, np.float32)
+    """The summation order is part of the definition.  Four blocks (one group,
+    zero-padded to 256): the pairwise tree adds (c0 + c2) + (c1 + c3) and keeps
+    both 2^-53 terms; a left-to-right sum loses each of them to round-to-even.
+    The float64 sums then fall on either side of a float32 midpoint of the mean:
+    tree -> 0.25 + 2^-25, left-to-right -> 0.25."""
+    c = np.array([1.0, 2.0 ** -53, 2.0 ** -24, 2.0 ** -53], np.float32)
     seq = 0.0
-    for v in c[:256]:
+    for v in c:
         seq += float(v)
-    tot = seq + float(np.float64(np.sum(c[256:], dtype=np.float64)))
-    assert nf4.fixed_order_mean(c) == np.float32(tot / c.size)
+    assert np.float32(seq / 4) == np.float32(0.25)
+    assert nf4.fixed_order_mean(c) == np.float32(0.25 + 2.0 ** -25)
 
 
 def test_double_quant_error_bound_and_format():
