@@ -66,4 +66,13 @@ __device__ __forceinline__ uint32_t bucket_code(float xh, const CodeBucket *tab)
   return static_cast<uint32_t>(e.base + (xh >= e.thr ? 1 : 0));
 }
 
+// Same lookup in a table replicated once per lane ([bucket][lane]), so that 32
+// lanes looking up arbitrary buckets never share a bank.
+__device__ __forceinline__ uint32_t lane_bucket_code(float xh, const CodeBucket (*tab)[32], int lane) {
+  int b = __float2int_rd(__fmaf_rn(xh, kBucketScale, kBucketScale));
+  b = min(max(b, 0), kBuckets - 1);
+  const CodeBucket e = tab[b][lane];
+  return static_cast<uint32_t>(e.base + (xh >= e.thr ? 1 : 0));
+}
+
 }  // namespace qlora

@@ -8,11 +8,11 @@
 //                          groups of 256 with one float32 scale per group.
 //
 // Three launches, all HBM-streaming and deterministic:
-//   k_quant_blocks : one CTA per group of 256 blocks.  8 threads per block, one
-//                    16-byte load each (all eight of a thread's loads issued
-//                    first); absmax by 3 xor-shuffles; exact quotient and code
-//                    via nf4_quant.cuh; nibble packing; per-group float64 sum of
-//                    the absmax values in block order (sequential, one thread).
+//   k_quant_blocks : CTAs walk the groups of 256 blocks, prefetching the next
+//                    group while coding the current one.  8 threads per block,
+//                    one 16-byte load each; absmax by 3 xor-shuffles; exact
+//                    quotient and code via nf4_quant.cuh; nibble packing;
+//                    per-group float64 pairwise tree of the absmax values.
 //   k_mean_tree    : one CTA, power-of-two pairwise tree over the group sums.
 //   k_double_quant : one CTA per group: centred constants, group absmax, S_g,
 //                    E4M3 codes (round to nearest even, saturating).
@@ -51,82 +51,105 @@ __device__ __forceinline__ uint4 ld_stream_v4(const void *p) {
 // path (exact there: see nf4_quant.cuh); smaller ones divide directly.
 constexpr float kFastQuotientMinAbsmax = 7.888609052210118e-31f;  // 2^-100
 
+// One CTA walks groups g = blockIdx.x, blockIdx.x + gridDim.x, ...; while it
+// codes one group the 16-byte loads of its next group are already in flight.
 __global__ void __launch_bounds__(256, 2) k_quant_blocks(const uint16_t *__restrict__ W, int64_t nb,
-                                                       uint8_t *__restrict__ codes, float *__restrict__ absmax,
-                                                       double *__restrict__ gsum, Nf4Thresholds thr,
-                                                       int *dev_err) {
-  __shared__ float s_amax[256];
-  __shared__ CodeBucket s_tab[kBuckets];
+                                                          uint8_t *__restrict__ codes, float *__restrict__ absmax,
+                                                          double *__restrict__ gsum, Nf4Thresholds thr,
+                                                          int *dev_err) {
+  __shared__ double s_sum[256];
+  __shared__ CodeBucket s_tab[kBuckets][32];  // one copy per lane: conflict-free random lookups
   pdl_launch_dependents();
-  if (threadIdx.x < kBuckets) s_tab[threadIdx.x] = make_bucket(threadIdx.x, thr.t);
-  const int64_t g = blockIdx.x;
+  for (int i = threadIdx.x; i < kBuckets * 32; i += 256) s_tab[i >> 5][i & 31] = make_bucket(i >> 5, thr.t);
+  const int64_t ng = (nb + 255) / 256;
   const int part = threadIdx.x & 7;  // 8-element chunk of the block
   const int sub = threadIdx.x >> 3;  // block within the pass
-  pdl_wait();
-  // all eight 16-byte loads of this thread in flight at once
-  uint4 raw[8];
+  const int lane = threadIdx.x & 31;
+  auto load_group = [&](int64_t g, uint4 (&raw)[8]) {
 #pragma unroll
-  for (int pass = 0; pass < 8; ++pass) {
-    const int64_t b = g * 256 + pass * 32 + sub;
-    raw[pass] = b < nb ? ld_stream_v4(W + b * 64 + part * 8) : make_uint4(0, 0, 0, 0);
-  }
+    for (int pass = 0; pass < 8; ++pass) {
+      const int64_t b = g * 256 + pass * 32 + sub;
+      raw[pass] = (g < ng && b < nb) ? ld_stream_v4(W + b * 64 + part * 8) : make_uint4(0, 0, 0, 0);
+    }
+  };
+  pdl_wait();
+  uint4 cur[8], nxt[8];
+  int64_t g = blockIdx.x;
+  load_group(g, cur);
   __syncthreads();  // bucket table ready
   bool bad = false;
+  for (; g < ng; g += gridDim.x) {
+    load_group(g + gridDim.x, nxt);
 #pragma unroll
-  for (int pass = 0; pass < 8; ++pass) {
-    const int lb = pass * 32 + sub;
-    const int64_t b = g * 256 + lb;
-    const bool valid = b < nb;
-    const uint32_t u[4] = {raw[pass].x, raw[pass].y, raw[pass].z, raw[pass].w};
-    float x[8];
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      x[2 * i] = __uint_as_float(u[i] << 16);
-      x[2 * i + 1] = __uint_as_float(u[i] & 0xFFFF0000u);
-    }
-    float amax = 0.f;
-#pragma unroll
-    for (int i = 0; i < 8; ++i) {
-      const float a = fabsf(x[i]);
-      bad |= !(a <= 3.402823466e38f);
-      amax = fmaxf(amax, a);
-    }
-    amax = fmaxf(amax, __shfl_xor_sync(0xFFFFFFFFu, amax, 1));
-    amax = fmaxf(amax, __shfl_xor_sync(0xFFFFFFFFu, amax, 2));
-    amax = fmaxf(amax, __shfl_xor_sync(0xFFFFFFFFu, amax, 4));
-    uint32_t packed = 0x77777777u;  // all-zero block: every code is the zero level
-    if (amax >= kFastQuotientMinAbsmax) {
-      const float ra = __frcp_rn(amax);
-      packed = 0;
+    for (int pass = 0; pass < 8; ++pass) {
+      const int lb = pass * 32 + sub;
+      const int64_t b = g * 256 + lb;
+      const bool valid = b < nb;
+      const uint32_t u[4] = {cur[pass].x, cur[pass].y, cur[pass].z, cur[pass].w};
+      float x[8];
 #pragma unroll
       for (int i = 0; i < 4; ++i) {
-        const uint32_t hi = bucket_code(quotient_rn(x[2 * i], amax, ra), s_tab);
-        const uint32_t lo = bucket_code(quotient_rn(x[2 * i + 1], amax, ra), s_tab);
-        packed |= ((hi << 4) | lo) << (8 * i);
+        x[2 * i] = __uint_as_float(u[i] << 16);
+        x[2 * i + 1] = __uint_as_float(u[i] & 0xFFFF0000u);
       }
-    } else if (amax > 0.f) {
-      packed = 0;
+      float amax = 0.f;
 #pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        const uint32_t hi = nf4_code(__fdiv_rn(x[2 * i], amax), thr);
-        const uint32_t lo = nf4_code(__fdiv_rn(x[2 * i + 1], amax), thr);
-        packed |= ((hi << 4) | lo) << (8 * i);
+      for (int i = 0; i < 8; ++i) {
+        const float av = fabsf(x[i]);
+        bad |= !(av <= 3.402823466e38f);
+        amax = fmaxf(amax, av);
       }
+      amax = fmaxf(amax, __shfl_xor_sync(0xFFFFFFFFu, amax, 1));
+      amax = fmaxf(amax, __shfl_xor_sync(0xFFFFFFFFu, amax, 2));
+      amax = fmaxf(amax, __shfl_xor_sync(0xFFFFFFFFu, amax, 4));
+      uint32_t packed = 0x77777777u;  // all-zero block: every code is the zero level
+      if (amax >= kFastQuotientMinAbsmax) {
+        const float ra = __frcp_rn(amax);
+        packed = 0;
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          const float xa = quotient_rn(x[2 * i], amax, ra);
+          const float xb = quotient_rn(x[2 * i + 1], amax, ra);
+          const uint32_t hi = lane_bucket_code(xa, s_tab, lane);
+          const uint32_t lo = lane_bucket_code(xb, s_tab, lane);
+          packed |= ((hi << 4) | lo) << (8 * i);
+        }
+      } else if (amax > 0.f) {
+        packed = 0;
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          const uint32_t hi = nf4_code(__fdiv_rn(x[2 * i], amax), thr);
+          const uint32_t lo = nf4_code(__fdiv_rn(x[2 * i + 1], amax), thr);
+          packed |= ((hi << 4) | lo) << (8 * i);
+        }
+      }
+      if (valid) {
+        reinterpret_cast<uint32_t *>(codes + b * 32)[part] = packed;
+        if (part == 0) absmax[b] = amax;
+      }
+      if (part == 0) s_sum[lb] = valid ? static_cast<double>(amax) : 0.0;
     }
-    if (valid) {
-      reinterpret_cast<uint32_t *>(codes + b * 32)[part] = packed;
-      if (part == 0) absmax[b] = amax;
+    // group sum: pairwise tree over the 256 (zero-padded) block constants
+    __syncthreads();
+    const int t = threadIdx.x;
+    for (int h = 128; h >= 32; h >>= 1) {
+      if (t < h) s_sum[t] = __dadd_rn(s_sum[t], s_sum[t + h]);
+      __syncthreads();
     }
-    if (part == 0) s_amax[lb] = valid ? amax : 0.f;
+    if (t < 32) {
+      double v = s_sum[t];
+#pragma unroll
+      for (int h = 16; h >= 1; h >>= 1) {
+        const double o = __shfl_down_sync(0xFFFFFFFFu, v, h);
+        if (t < h) v = __dadd_rn(v, o);
+      }
+      if (t == 0) gsum[g] = v;
+    }
+    __syncthreads();  // s_sum is reused by the next group
+#pragma unroll
+    for (int pass = 0; pass < 8; ++pass) cur[pass] = nxt[pass];
   }
   if (bad && dev_err) atomicOr(dev_err, QLORA_DEVERR_NONFINITE);
-  __syncthreads();
-  if (threadIdx.x == 0) {
-    const int64_t cnt = nb - g * 256 < 256 ? nb - g * 256 : 256;
-    double acc = 0.0;
-    for (int j = 0; j < cnt; ++j) acc = __dadd_rn(acc, static_cast<double>(s_amax[j]));
-    gsum[g] = acc;
-  }
 }
 
 // Pairwise tree over the power-of-two padded group sums: for h = size/2, ..., 1
@@ -216,7 +239,10 @@ cudaError_t launch_quantize(const uint16_t *W, int64_t nb, uint8_t *codes, uint8
                             float *ws_absmax, double *ws_gsum, int64_t gsum_size, const Nf4Thresholds &thr,
                             int *dev_err, cudaStream_t st) {
   const int64_t ng = (nb + 255) / 256;
-  cudaError_t e = launch_k(k_quant_blocks, dim3(static_cast<unsigned>(ng)), dim3(256), 0, st, 1, W, nb, codes,
+  int dev = 0, sms = 148;
+  if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  const int64_t grid = ng < 2 * static_cast<int64_t>(sms) ? ng : 2 * static_cast<int64_t>(sms);
+  cudaError_t e = launch_k(k_quant_blocks, dim3(static_cast<unsigned>(grid)), dim3(256), 0, st, 1, W, nb, codes,
                            ws_absmax, ws_gsum, thr, dev_err);
   if (e != cudaSuccess) return e;
   e = launch_k(k_mean_tree, dim3(1), dim3(1024), 0, st, 1, ws_gsum, ng, gsum_size, nb, mean);
