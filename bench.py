@@ -16,6 +16,8 @@ slowest rank's time (weak scaling).  Rank 0 prints one JSON line.
 from __future__ import annotations
 
 import argparse
+import datetime
+import hashlib
 import json
 import os
 import statistics
@@ -42,9 +44,26 @@ def _peaks():
         return 6650.0, 1590.0, 1400.0, "fallback"
 
 
+# DRAM traffic (read + write bytes per launch) of the fused dequant GEMMs from the
+# ncu capture summarised in profiles/fused_dequant_gemm_proj7b.md.  Reported only
+# while the kernel sources hash to the build that capture was taken of.
+KERNEL_SOURCES = ["gemm_pair.cuh", "gemm.cuh", "nf4_decode.cuh", "ptx.cuh", "launch.cuh", "linear.cu"]
+TRAFFIC_CAPTURE = {"sources_sha1": "9e76271469033462adef098d70f711f9df8b8dd8",
+                   "fwd_y": 49_781_000, "bwd_dx": 47_768_000}
+
+
+def kernel_sources_sha1() -> str:
+    h = hashlib.sha1()
+    for f in KERNEL_SOURCES:
+        with open(os.path.join(ROOT, "bit_nf4_quantised_codebook_b200", "csrc", f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()
+
+
 class ClockSampler:
-    """nvidia-smi clocks / throttle reasons sampled while the timed region runs."""
-    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+    """nvidia-smi clocks / throttle reasons sampled while the timed region runs;
+    only samples stamped inside [mark_start, mark_end] are kept."""
+    FIELDS = ("timestamp,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
               "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
 
@@ -52,6 +71,14 @@ class ClockSampler:
         self.gpu_id = gpu_id
         self.proc = None
         self.path = None
+        self.t0 = None
+        self.t1 = None
+
+    def mark_start(self):
+        self.t0 = datetime.datetime.now()
+
+    def mark_end(self):
+        self.t1 = datetime.datetime.now()
 
     def start(self):
         try:
@@ -74,19 +101,29 @@ class ClockSampler:
             self.proc.wait(timeout=5)
         except Exception:
             self.proc.kill()
-        rows = []
+        rows, all_rows = [], []
         with open(self.path) as f:
             for ln in f:
                 parts = [p.strip() for p in ln.split(",")]
-                if len(parts) >= 9:
+                if len(parts) < 9:
+                    continue
+                all_rows.append(parts)
+                try:
+                    ts = datetime.datetime.strptime(parts[0], "%Y/%m/%d %H:%M:%S.%f")
+                except ValueError:
+                    continue
+                if self.t0 and self.t1 and self.t0 <= ts <= self.t1:
                     rows.append(parts)
         os.unlink(self.path)
+        if not rows:  # timed region shorter than the sampling period: keep the nearest samples
+            rows = all_rows[-3:]
         sm = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
         mx = [float(r[2]) for r in rows if r[2].replace(".", "").isdigit()]
         names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
         reasons = sorted({names[i] for r in rows for i in range(4) if r[5 + i].lower() == "active"})
         return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(mx) if mx else None,
-                "reasons": reasons, "samples": len(rows)}
+                "reasons": reasons, "samples": len(rows),
+                "power_w_max": max((float(r[3]) for r in rows if r[3].replace(".", "").isdigit()), default=None)}
 
 
 def _dist():
@@ -165,6 +202,7 @@ def run_ours(args):
         dist.barrier()
     torch.cuda.synchronize()
     launches0 = api.qlora_kernel_launch_count()
+    sampler.mark_start()
     t0 = torch.cuda.Event(enable_timing=True)
     t1 = torch.cuda.Event(enable_timing=True)
     t0.record()
@@ -173,6 +211,7 @@ def run_ours(args):
         step(i)
     t1.record()
     torch.cuda.synchronize()
+    sampler.mark_end()
     api.qlora_set_timing_events()
     launches = api.qlora_kernel_launch_count() - launches0
     if world > 1:
@@ -229,6 +268,9 @@ def run_ours(args):
     dom_flops = 2.0 * M * N * K + 2.0 * M * r * (K if dom == "bwd_dx" else N)
     achieved = dom_flops / (dom_ms * 1e-3) / 1e12
     packed = wq.nbytes()
+    traffic = None
+    if TRAFFIC_CAPTURE["sources_sha1"] and TRAFFIC_CAPTURE["sources_sha1"] == kernel_sources_sha1():
+        traffic = TRAFFIC_CAPTURE.get(dom)
 
     line = {
         "metric": METRIC, "value": round(value, 3), "unit": "TFLOP/s", "n_gpus": world,
@@ -244,7 +286,7 @@ def run_ours(args):
         "roofline": {"kernel": f"fused dequant GEMM ({dom})", "bound": "tensor",
                      "achieved": round(achieved, 2), "peak": bf16_burst, "unit": "TFLOP/s",
                      "frac": round(achieved / bf16_burst, 4), "peak_source": f"{peak_src} bf16 burst",
-                     "traffic": None},
+                     "traffic": traffic, "traffic_unit": "bytes per launch (ncu dram read+write)"},
         "e2e": {"value": round(e2e_value, 3), "unit": "TFLOP/s", "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h, "steps": e2e_steps},
         "gpu_launches": int(launches),
@@ -279,11 +321,19 @@ def _oracle_sample(rows: int, qrows: int | None = None):
     return dt, c.flops_fwd() + c.flops_bwd()
 
 
-def cpu_baseline(rows: int = 256) -> dict:
-    dt, fl = _oracle_sample(rows)
-    return {"value": round(fl / dt / 1e12, 6), "unit": "TFLOP/s", "cores": os.cpu_count(), "kind": "oracle",
-            "sample": f"quantise+dequantise the full 4096x4096 W, fwd+bwd on {rows} of 4096 token rows "
-                      f"(float64 numpy, BLAS threads = cores); {dt:.1f} s"}
+def cpu_baseline(min_seconds: float = 10.0) -> dict:
+    """The oracle as it stands on the full workload (quantise + dequantise the
+    4096 x 4096 W, forward + backward on all 4096 token rows), repeated until
+    `min_seconds` of host time have passed."""
+    tot_t, tot_f, n = 0.0, 0.0, 0
+    while tot_t < min_seconds or n == 0:
+        dt, fl = _oracle_sample(4096)
+        tot_t += dt
+        tot_f += fl
+        n += 1
+    return {"value": round(tot_f / tot_t / 1e12, 6), "unit": "TFLOP/s", "cores": os.cpu_count(), "kind": "oracle",
+            "sample": f"{n} x the full step on the host (quantise + dequantise the 4096x4096 W, fwd + bwd on "
+                      f"4096 tokens; float64 numpy, BLAS threads = cores); {tot_t:.1f} s"}
 
 
 def run_reference(args):
