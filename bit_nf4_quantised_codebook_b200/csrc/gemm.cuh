@@ -152,8 +152,8 @@ __global__ void __launch_bounds__(C::NUM_THREADS, 1)
   tc_fence_after();
   const uint32_t tmem_acc = *tmem_slot;
   const uint32_t smem_base = smem_u32(smem);
-  pdl_launch_dependents();
   pdl_wait();  // inputs of this grid were written by earlier grids of the stream
+  pdl_launch_dependents();
 
   if (warp == 0) {
     // ------------------------------------------------------------ TMA producer

@@ -1,10 +1,13 @@
 // launch.cuh — every kernel of the library is launched through launch_k():
 // cudaLaunchKernelEx with programmatic dependent launch enabled (and, for the
-// skinny GEMMs, a 1 x 1 x cz cluster).  Each kernel calls pdl_launch_dependents()
-// once its CTAs are running and pdl_wait() before its first access to global
-// memory, so the next kernel's CTAs can be placed and run their prologue
-// (barrier init, TMEM allocation, tensor-map prefetch) while the previous
-// kernel drains; stream order for memory is unchanged.
+// skinny GEMMs, a 1 x 1 x cz cluster).  Each kernel calls pdl_wait() before its
+// first access to global memory and pdl_launch_dependents() right after it, so
+// the next kernel's CTAs can be placed and run their prologue (barrier init,
+// TMEM allocation, tensor-map prefetch) while this one runs; stream order for
+// memory is unchanged.  Because a kernel triggers its dependents only after its
+// own wait returned, every grid before its predecessor is complete when a
+// dependent starts: a dependent that reads some inputs before its own wait may
+// rely on that (it must still wait before reading its predecessor's output).
 #pragma once
 #include <utility>
 #include <cuda_runtime.h>

@@ -88,8 +88,8 @@ static cudaError_t launch_pair(dim3 grid, const TmaMaps &m, const GemmParams &p,
 // out[row, c] = cvt(scale * sum_s part[s][row][c]), c < cols, sequential over s.
 __global__ void k_finalize_bf16(const float *__restrict__ part, int splits, int64_t split_stride, int64_t rows,
                                 int cols, int ldp, float scale, uint16_t *__restrict__ out, int64_t ldo) {
-  pdl_launch_dependents();
   pdl_wait();
+  pdl_launch_dependents();
   const int64_t idx = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
   const int64_t nvec = rows * (cols / 4);
   if (idx >= nvec) return;

@@ -59,7 +59,6 @@ __global__ void __launch_bounds__(256, 2) k_quant_blocks(const uint16_t *__restr
                                                           int *dev_err) {
   __shared__ double s_sum[256];
   __shared__ CodeBucket s_tab[kBuckets][32];  // one copy per lane: conflict-free random lookups
-  pdl_launch_dependents();
   for (int i = threadIdx.x; i < kBuckets * 32; i += 256) s_tab[i >> 5][i & 31] = make_bucket(i >> 5, thr.t);
   const int64_t ng = (nb + 255) / 256;
   const int part = threadIdx.x & 7;  // 8-element chunk of the block
@@ -73,6 +72,7 @@ __global__ void __launch_bounds__(256, 2) k_quant_blocks(const uint16_t *__restr
     }
   };
   pdl_wait();
+  pdl_launch_dependents();
   uint4 cur[8], nxt[8];
   int64_t g = blockIdx.x;
   load_group(g, cur);
@@ -159,8 +159,8 @@ __global__ void __launch_bounds__(256, 2) k_quant_blocks(const uint16_t *__restr
 __global__ void __launch_bounds__(1024) k_mean_tree(double *__restrict__ a, int64_t ng, int64_t size, int64_t nb,
                                                      float *__restrict__ mean) {
   __shared__ double s[1024];
-  pdl_launch_dependents();
   pdl_wait();
+  pdl_launch_dependents();
   for (int64_t i = ng + threadIdx.x; i < size; i += blockDim.x) a[i] = 0.0;
   __syncthreads();
   int64_t h = size / 2;
@@ -191,8 +191,8 @@ __global__ void __launch_bounds__(256) k_double_quant(const float *__restrict__ 
                                                        const float *__restrict__ mean, uint8_t *__restrict__ c2q,
                                                        float *__restrict__ c1) {
   __shared__ float s_red[8];
-  pdl_launch_dependents();
   pdl_wait();
+  pdl_launch_dependents();
   const int64_t g = blockIdx.x;
   const int64_t b = g * 256 + threadIdx.x;
   const bool valid = b < nb;
@@ -216,8 +216,8 @@ __global__ void __launch_bounds__(256) k_double_quant(const float *__restrict__ 
 __global__ void __launch_bounds__(256) k_dequant(const uint8_t *__restrict__ codes, const uint8_t *__restrict__ c2q,
                                                   const float *__restrict__ c1, const float *__restrict__ mean,
                                                   int64_t nb, Nf4Levels lv, uint16_t *__restrict__ out) {
-  pdl_launch_dependents();
   pdl_wait();
+  pdl_launch_dependents();
   const int64_t b = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
   if (b >= nb) return;
   const float c2h = reconstruct_c2(c2q[b], c1[b >> 8], *mean);
