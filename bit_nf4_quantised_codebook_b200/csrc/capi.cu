@@ -64,7 +64,6 @@ bool encode_2d(CUtensorMap *m, CUtensorMapDataType dt, const void *ptr, uint64_t
             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-int ceil_div(int64_t a, int64_t b) { return static_cast<int>((a + b - 1) / b); }
 
 SplitPlan choose(int64_t tiles, int64_t k_total, int target_ctas, int min_iters) {
   SplitPlan sp;
@@ -87,6 +86,29 @@ SplitPlan choose_cluster(int64_t tiles, int64_t k_total, int target_ctas) {
   sp.splits = s;
   sp.k_iters = static_cast<int>((k_total + s - 1) / s);
   return sp;
+}
+
+// K splits of the small-M forward (one cluster of S <= 8 CTAs per 128 W rows):
+// minimise waves x steps per split over 2 CTAs per SM, ties to fewer splits.
+SplitPlan choose_small(int64_t N, int64_t k_total, int num_sms) {
+  SplitPlan best;
+  best.k_iters_total = static_cast<int>(k_total);
+  const int64_t tiles = (N + 127) / 128, slots = 2 * static_cast<int64_t>(num_sms);
+  int64_t best_cost = -1;
+  for (int s = 1; s <= 8; ++s) {
+    int64_t kps = (k_total + s - 1) / s;
+    if (k_total % 4 == 0) kps = (kps + 3) / 4 * 4;  // splits start on 4-byte boundaries of a constants row
+    if (kps > kSmallMaxKIters) continue;
+    if (s > 1 && (s - 1) * kps >= k_total) continue;  // a split would have no work
+    const int64_t waves = (tiles * s + slots - 1) / slots;
+    const int64_t cost = waves * kps;
+    if (best_cost < 0 || cost < best_cost) {
+      best_cost = cost;
+      best.splits = s;
+      best.k_iters = static_cast<int>(kps);
+    }
+  }
+  return best;
 }
 
 size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
@@ -156,6 +178,12 @@ LinearPlan make_plan(int op, int64_t M, int64_t N, int64_t K, int r, int num_sms
   pl.sp_t = choose_cluster(mt, K / 64, 2 * num_sms);
   pl.off_sT = take(static_cast<size_t>(M) * r * 2);
   if (op == QLORA_OP_FORWARD) {
+    if (M <= kSmallMaxTokens && K / 64 <= 8 * kSmallMaxKIters) {
+      pl.small_main = true;
+      pl.sp_main = choose_small(N, K / 64, num_sms);
+      pl.bytes = off;
+      return pl;
+    }
     pl.pair_main = M > 128;
     pl.sp_main = choose((pl.pair_main ? 2 * ((M + 511) / 512) : mt) * ((N + 255) / 256), K / 64, num_sms, 4);
     if (pl.sp_main.splits > 1) pl.off_main_part = take(static_cast<size_t>(pl.sp_main.splits) * M * N * 4);
@@ -180,9 +208,12 @@ bool map_bf16_mn(CUtensorMap *m, const void *ptr, int64_t inner, int64_t outer) 
   return encode_2d(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, ptr, inner, outer, inner * 2, 64, 64,
                    CU_TENSOR_MAP_SWIZZLE_128B);
 }
-bool map_codes(CUtensorMap *m, const void *codes, int64_t N, int64_t K, int box_bytes, int box_rows, bool swizzle64) {
-  return encode_2d(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, codes, K / 2, N, K / 2, box_bytes, box_rows,
-                   swizzle64 ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_NONE);
+bool map_codes(CUtensorMap *m, const void *codes, int64_t N, int64_t K, int box_bytes, int box_rows,
+               int swizzle_bytes) {
+  const CUtensorMapSwizzle sw = swizzle_bytes == 64   ? CU_TENSOR_MAP_SWIZZLE_64B
+                                : swizzle_bytes == 32 ? CU_TENSOR_MAP_SWIZZLE_32B
+                                                      : CU_TENSOR_MAP_SWIZZLE_NONE;
+  return encode_2d(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, codes, K / 2, N, K / 2, box_bytes, box_rows, sw);
 }
 
 }  // namespace qlora

@@ -20,6 +20,7 @@
 #include <cuda_runtime.h>
 #include "gemm.cuh"
 #include "gemm_pair.cuh"
+#include "gemm_smallm.cuh"
 #include "internal.h"
 #include "launch.cuh"
 #include "linear_plan.h"
@@ -185,9 +186,9 @@ static cudaError_t run_fused(bool fwd, const LaunchCtx &c, const qlora_nf4_weigh
   TmaMaps m;
   bool ok = map_bf16_kmajor(&m.a, act, red, M, 128) && map_bf16_kmajor(&m.a2, lora_a, r, M, 128);
   if (fwd) {
-    ok = ok && map_codes(&m.b, w.codes, N, K, 32, pair ? 128 : 256, false) && map_bf16_mn(&m.b2, lora_b, N, r);
+    ok = ok && map_codes(&m.b, w.codes, N, K, 32, pair ? 128 : 256, 0) && map_bf16_mn(&m.b2, lora_b, N, r);
   } else {
-    ok = ok && (pair ? map_codes(&m.b, w.codes, N, K, 64, 64, true) : map_codes(&m.b, w.codes, N, K, 128, 64, false)) &&
+    ok = ok && (pair ? map_codes(&m.b, w.codes, N, K, 64, 64, 64) : map_codes(&m.b, w.codes, N, K, 128, 64, 0)) &&
          map_bf16_kmajor(&m.b2, lora_b, r, K, pair ? 128 : 256);
   }
   if (!ok) return cudaErrorInvalidValue;
@@ -223,6 +224,71 @@ static cudaError_t run_fused(bool fwd, const LaunchCtx &c, const qlora_nf4_weigh
   return cudaSuccess;
 }
 
+// ---------------------------------------------------------------- small-M forward
+#ifndef QLORA_SMALL_GROUPS
+#define QLORA_SMALL_GROUPS 2
+#endif
+constexpr int kSmallGroups = QLORA_SMALL_GROUPS;  // dequant groups of 4 warps per CTA
+
+template <class C>
+static cudaError_t launch_small(dim3 grid, int cz, const TmaMaps &m, const SmallParams &p, cudaStream_t st) {
+  static bool prepared = false;
+  if (!prepared) {
+    cudaError_t e = cudaFuncSetAttribute(gemm_smallm_kernel<C>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         C::SMEM_BYTES);
+    if (e != cudaSuccess) return e;
+    prepared = true;
+  }
+  return launch_k(gemm_smallm_kernel<C>, grid, dim3(C::NUM_THREADS), C::SMEM_BYTES, st, static_cast<unsigned>(cz),
+                  m.a, m.b, m.a2, m.b2, p);
+}
+
+// Y = X·W_hatᵀ + sT·B for M <= 64 tokens: W rows on the MMA M side, tokens on N.
+static cudaError_t run_small_forward(const LaunchCtx &c, const qlora_nf4_weight &w, const uint16_t *X, int64_t M,
+                                     const uint16_t *sT, const uint16_t *B, int r, uint16_t *Y, const SplitPlan &sp,
+                                     cudaEvent_t ev0, cudaEvent_t ev1) {
+  const int N = static_cast<int>(w.N), K = static_cast<int>(w.K);
+  const int nt = static_cast<int>((M + 15) / 16) * 16;
+  TmaMaps m;  // a = X, b = codes, a2 = sT, b2 = B
+  if (!map_bf16_kmajor(&m.a, X, K, M, nt) || !map_codes(&m.b, w.codes, N, K, 64, 128, 64) ||
+      !map_bf16_kmajor(&m.a2, sT, r, M, nt) || !map_bf16_mn(&m.b2, B, N, r))
+    return cudaErrorInvalidValue;
+  SmallParams p;
+  std::memset(&p, 0, sizeof(p));
+  p.M = static_cast<int>(M);
+  p.N = N;
+  p.k_iters = sp.k_iters;
+  p.k_iters_total = sp.k_iters_total;
+  p.splits = sp.splits;
+  int words = (sp.k_iters + 3) / 4;
+  if (words % 2 == 0) ++words;  // odd word stride: 32 consecutive rows hit 32 banks
+  p.q8_stride = 4 * words;
+  p.q8_words = (sp.k_iters_total % 4 == 0 && sp.k_iters % 4 == 0) ? 1 : 0;
+  p.lora_r = r;
+  p.c2q = w.c2q;
+  p.c1 = w.c1;
+  p.mean = w.mean;
+  p.lv = c.levels;
+  p.k_shr16 = 1u << 16;
+  p.k_shr1 = 1u << 31;
+  p.Y = Y;
+  p.dev_err = c.dev_err;
+  p.timeout_ns = c.timeout_ns;
+  const dim3 grid(static_cast<unsigned>((N + 127) / 128), 1, static_cast<unsigned>(sp.splits));
+  if (ev0) cudaEventRecord(ev0, c.stream);
+  cudaError_t e;
+  switch (nt) {
+    case 16: e = launch_small<SmallCfg<16, kSmallGroups>>(grid, sp.splits, m, p, c.stream); break;
+    case 32: e = launch_small<SmallCfg<32, kSmallGroups>>(grid, sp.splits, m, p, c.stream); break;
+    case 48: e = launch_small<SmallCfg<48, kSmallGroups>>(grid, sp.splits, m, p, c.stream); break;
+    case 64: e = launch_small<SmallCfg<64, kSmallGroups>>(grid, sp.splits, m, p, c.stream); break;
+    default: return cudaErrorInvalidValue;
+  }
+  if (e != cudaSuccess) return e;
+  if (ev1) cudaEventRecord(ev1, c.stream);
+  return cudaSuccess;
+}
+
 // ---------------------------------------------------------------- forward
 // sT = bf16(s·X·A)  (A-op X [M,K] K-major; B-op Aᵀ: A [K,r] read MN-major)
 static cudaError_t run_t(const LaunchCtx &c, const uint16_t *X, int64_t M, int K, const uint16_t *A, int r, float s,
@@ -243,6 +309,7 @@ cudaError_t run_forward(const LaunchCtx &c, const qlora_nf4_weight &w, const uin
   if ((e = run_t(c, X, M, K, A, r, s, sT, pl)) != cudaSuccess) return e;
   // Y = X·W_hatᵀ + sT·B
   const TimingHooks &hk = timing_hooks();
+  if (pl.small_main) return run_small_forward(c, w, X, M, sT, B, r, Y, pl.sp_main, hk.fwd_begin, hk.fwd_end);
   float *part = reinterpret_cast<float *>(ws + pl.off_main_part);
   return run_fused(true, c, w, X, M, sT, B, r, Y, pl.pair_main, pl.sp_main, part, hk.fwd_begin, hk.fwd_end);
 }

@@ -21,6 +21,12 @@ struct LaunchCtx {
   Nf4Levels levels;
 };
 
+// Forward at M <= kSmallMaxTokens runs the swapped-orientation kernel
+// (gemm_smallm.cuh): K splits of at most kSmallMaxKIters steps, at most 8 per
+// cluster, so K <= 8 · 64 · kSmallMaxKIters.
+constexpr int kSmallMaxTokens = 64;
+constexpr int kSmallMaxKIters = 64;
+
 struct SplitPlan {
   int splits = 1;
   int k_iters = 0;        // stages per split
@@ -31,6 +37,7 @@ struct LinearPlan {
   int rpad = 16;
   SplitPlan sp_t, sp_u, sp_main, sp_dx, sp_da, sp_db;
   bool pair_main = false, pair_dx = false;  // CTA-pair kernel for the fused GEMMs
+  bool small_main = false;                  // forward through the small-M kernel (sp_main = its splits)
   size_t off_sT = 0, off_sU = 0, off_main_part = 0;
   size_t off_absmax = 0, off_gsum = 0;
   int64_t gsum_size = 0;
@@ -44,8 +51,9 @@ LinearPlan make_plan(int op, int64_t M, int64_t N, int64_t K, int r, int num_sms
 bool map_bf16_kmajor(CUtensorMap *m, const void *ptr, int64_t inner, int64_t outer, int box_rows);
 // bf16 [outer, inner] row-major, read MN-major (inner = MN): box {64, 64}, 128-byte swizzle.
 bool map_bf16_mn(CUtensorMap *m, const void *ptr, int64_t inner, int64_t outer);
-// packed codes of an N x K weight, uint8 [N, K/2]: box {box_bytes, box_rows}, no swizzle or the 64-byte swizzle.
-bool map_codes(CUtensorMap *m, const void *codes, int64_t N, int64_t K, int box_bytes, int box_rows, bool swizzle64);
+// packed codes of an N x K weight, uint8 [N, K/2]: box {box_bytes, box_rows}; swizzle_bytes 0 (none), 32 or 64.
+bool map_codes(CUtensorMap *m, const void *codes, int64_t N, int64_t K, int box_bytes, int box_rows,
+               int swizzle_bytes);
 
 cudaError_t run_forward(const LaunchCtx &c, const qlora_nf4_weight &w, const uint16_t *X, int64_t M,
                         const uint16_t *A, const uint16_t *B, int r, float s, uint16_t *Y, uint16_t *T_save,

@@ -105,6 +105,21 @@ def test_small_m_forward(m):
     assert_close(bf16_f64(sT), case.s * ref["T"], f"sT[m={m}]")
 
 
+@pytest.mark.parametrize("m,n,k,r", [
+    (1, 264, 320, 24),     # ragged W-row tile, 5 K steps, one partial adapter chunk
+    (17, 1000, 4096, 136), # 32-token tile, 3 adapter chunks (64 + 64 + 8)
+    (33, 512, 32768, 64),  # 48-token tile, the longest K of this path (8 splits x 64 steps)
+    (64, 256, 64, 8),      # one K step, no split
+    (48, 8, 128, 16),      # fewer W rows than one tile
+])
+def test_small_m_path_edges(m, n, k, r):
+    """Forward at M <= 64 (W rows on the MMA M side, tokens on N): ragged tiles,
+    K-split counts and adapter ranks; backward on the same data."""
+    case = inputs.LinearCase(f"smallm_edge_{m}x{n}x{k}_r{r}", M=m, N=n, K=k, r=r, alpha=16.0, w_std=0.02,
+                             a_std=0.05, b_std=0.05, seed=11 + m)
+    _run(case)
+
+
 def test_proj7b_full_size_sampled():
     """The 4096^3 projection in the benchmark's launch configuration: sampled
     token rows of Y and dX, full dA and dB."""
