@@ -97,6 +97,7 @@ struct GemmCfg {
   static_assert(BN % 16 == 0 && BN >= 16 && BN <= 256, "UMMA N");
   static_assert(!DQ || BN == 256, "dequant tiles are 256 wide");
   static_assert(STAGE_BYTES % 1024 == 0, "swizzle atoms need 1 KiB alignment");
+  static_assert((3 * STAGES + 2) * 8 <= BAR_BYTES, "barriers, TMEM slot and abort flag fit");
 };
 
 template <class C>
