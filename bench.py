@@ -1,6 +1,7 @@
 """Benchmark of the QLoRA frozen-NF4 linear layer on B200.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+                    [--workload proj7b | smallm --n N --m M]
 
 One step = the whole hot path on one batch: NF4 + double quantisation of the
 bf16 weight, the forward (T = X·A, fused dequant GEMM Y = X·W_hatᵀ + sT·B) and
@@ -8,6 +9,11 @@ the backward (U = dY·Bᵀ, fused dequant GEMM dX = dY·W_hat + sU·Aᵀ, dA, dB
 Workload: a single 7B-class projection, W 4096 x 4096, X 4096 tokens
 (batch 4 x seq 1024), LoRA r = 64, alpha = 16, synthetic seeded inputs.
 value = algorithmic fwd+bwd flops per step / device time (TFLOP/s).
+
+--workload smallm: the decode-sized forward (K = 8192, N = 8192 or 28672 W rows,
+M = 1..64 tokens, r = 64; the weight quantised once and resident, rotated over
+enough copies to exceed L2); value = packed-weight bytes streamed per forward /
+device time (GB/s).
 
 Multi-GPU: the layer does not shard (one GPU per replica), so every rank runs
 its own replica of the workload and value sums the replicas' work over the
@@ -48,8 +54,8 @@ def _peaks():
 # ncu capture summarised in profiles/fused_dequant_gemm_proj7b.md.  Reported only
 # while the kernel sources hash to the build that capture was taken of.
 KERNEL_SOURCES = ["gemm_pair.cuh", "gemm.cuh", "nf4_decode.cuh", "ptx.cuh", "launch.cuh", "linear.cu"]
-TRAFFIC_CAPTURE = {"sources_sha1": "9e76271469033462adef098d70f711f9df8b8dd8",
-                   "fwd_y": 49_781_000, "bwd_dx": 47_768_000}
+TRAFFIC_CAPTURE = {"sources_sha1": "3abf9dad4be07b23c132b3cb417859c219552969",
+                   "fwd_y": 46_942_976, "bwd_dx": 45_571_072}
 
 
 def kernel_sources_sha1() -> str:
@@ -301,6 +307,150 @@ def run_ours(args):
         dist.destroy_process_group()
 
 
+def run_smallm(args):
+    """Forward only at decode batch sizes: T = X·A, then the small-M dequant GEMM."""
+    import torch
+    import torch.distributed as dist
+    from datetime import timedelta
+    from bit_nf4_quantised_codebook_b200 import api, inputs
+
+    world, rank, local = _dist()
+    torch.cuda.set_device(local)
+    if world > 1:
+        dist.init_process_group("nccl", timeout=timedelta(seconds=120), device_id=torch.device("cuda", local))
+    api.lib()
+    dev = torch.device("cuda", local)
+    case = inputs.small_m(args.n, args.m)
+    M, N, K, r, s = case.M, case.N, case.K, case.r, case.s
+    W = api.bits_to_tensor(case.W(), dev)
+    ncopy = max(2, -(-3 * 128 * 2**20 // (N * K // 2)))  # weight copies: > 3x L2 in total
+    qs = [api.qlora_quantize(W) for _ in range(ncopy)]
+    del W
+    packed = qs[0].nbytes()
+    X, A, B = (api.bits_to_tensor(getattr(case, k)(), dev) for k in ("X", "A", "B"))
+    Y = torch.empty(M, N, dtype=torch.bfloat16, device=dev)
+    sT = torch.empty(M, r, dtype=torch.bfloat16, device=dev)
+    ws = torch.empty(max(1, api.qlora_workspace_size(api.QLORA_OP_FORWARD, M, N, K, r)), dtype=torch.uint8,
+                     device=dev)
+    err = api.new_error_word(dev)
+
+    def step(i, Xin=None):
+        api.qlora_linear_forward(qs[i % ncopy], X if Xin is None else Xin, A, B, s, Y=Y, T_save=sT, ws=ws,
+                                 dev_err=err)
+
+    for i in range(args.warmup):
+        step(i)
+    torch.cuda.synchronize()
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(args.steps)]
+    for pair in ev:
+        for e in pair:
+            e.record()
+    gpu_id = None
+    try:
+        gpu_id = "GPU-" + str(torch.cuda.get_device_properties(local).uuid)
+    except Exception:
+        pass
+    sampler = ClockSampler(gpu_id)
+    sampler.start()
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    launches0 = api.qlora_kernel_launch_count()
+    sampler.mark_start()
+    t0 = torch.cuda.Event(enable_timing=True)
+    t1 = torch.cuda.Event(enable_timing=True)
+    t0.record()
+    for i in range(args.steps):
+        step(i)
+    t1.record()
+    torch.cuda.synchronize()
+    sampler.mark_end()
+    launches = api.qlora_kernel_launch_count() - launches0
+    # the dominant kernel alone: events around it (they end the programmatic overlap
+    # with the X·A kernel, so this loop is timed separately from the step loop)
+    for i in range(args.steps):
+        api.qlora_set_timing_events(ev[i][0], ev[i][1])
+        step(i)
+    torch.cuda.synchronize()
+    api.qlora_set_timing_events()
+    clocks = sampler.stop()
+    ms = t0.elapsed_time(t1)
+    kern_ms = sum(a.elapsed_time(b) for a, b in ev) / args.steps
+    if world > 1:
+        t = torch.tensor([ms], device=dev, dtype=torch.float64)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms = float(t.item())
+    if int(err[0].item()) != 0:
+        raise RuntimeError(f"device error word {int(err[0].item())}")
+    ms_step = ms / args.steps
+    value = packed * world / (ms_step * 1e-3) / 1e9
+
+    # end to end: X host -> device, forward, Y device -> host
+    e2e_steps = max(3, min(100, args.steps // 10))
+    hx = X.cpu().pin_memory()
+    hy = torch.empty_like(Y, device="cpu").pin_memory()
+    dx = torch.empty_like(X)
+    torch.cuda.synchronize()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for i in range(e2e_steps):
+        dx.copy_(hx, non_blocking=True)
+        step(i, dx)
+        hy.copy_(Y, non_blocking=True)
+    e1.record()
+    torch.cuda.synchronize()
+    e2e_ms = e0.elapsed_time(e1) / e2e_steps
+
+    hbm, _, _, peak_src = _peaks()
+    achieved = packed / (kern_ms * 1e-3) / 1e9
+    line = {
+        "metric": METRIC, "value": round(value, 2), "unit": "GB/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_step, 5),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic (seeded numpy N(0,std) rounded to bf16)",
+        "config": {"workload": f"small-M forward: W {N}x{K} NF4+DQ, {M} tokens, LoRA r={r} alpha={case.alpha}",
+                   "M": M, "N": N, "K": K, "r": r, "parallelism": f"replicas x{world} (no shard)",
+                   "step": "forward (X·A, then the dequant GEMM with the adapter term)",
+                   "l2": f"{ncopy} resident weight copies used in rotation ({ncopy * packed / 1e6:.0f} MB > L2)"},
+        "kernels": {"smallm_gemm_ms": round(kern_ms, 5)},
+        "roofline": {"kernel": "small-M dequant GEMM", "bound": "hbm", "achieved": round(achieved, 1),
+                     "peak": hbm, "unit": "GB/s", "frac": round(achieved / hbm, 4),
+                     "peak_source": f"{peak_src} HBM copy", "traffic": None,
+                     "traffic_unit": "bytes per launch (ncu dram read+write)"},
+        "e2e": {"value": round(packed / (e2e_ms * 1e-3) / 1e9, 2), "unit": "GB/s",
+                "h2d_bytes_per_step": X.numel() * 2, "d2h_bytes_per_step": Y.numel() * 2, "steps": e2e_steps},
+        "gpu_launches": int(launches),
+        "clocks": clocks,
+    }
+    if world == 1 and rank == 0 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline_smallm(case)
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+def cpu_baseline_smallm(case, min_seconds: float = 10.0) -> dict:
+    """The oracle on a slice of the small-M forward: quantise `rows` W rows and run
+    the forward for all tokens through them; GB/s of packed weight per host second."""
+    from oracle import linear, nf4
+    rows = 256
+    W, X, A, B = case.W()[:rows], case.X(), case.A(), case.B()[:, :rows]
+    tot_t, n = 0.0, 0
+    while tot_t < min_seconds or n == 0:
+        t = time.perf_counter()
+        what = nf4.dequantize_nf4(nf4.quantize_nf4(W))
+        linear.forward(X, what, A, B, case.s)
+        tot_t += time.perf_counter() - t
+        n += 1
+    packed = rows * case.K // 2 + rows * case.K // 64
+    return {"value": round(n * packed / tot_t / 1e9, 6), "unit": "GB/s", "cores": os.cpu_count(), "kind": "oracle",
+            "sample": f"{n} x (quantise + dequantise {rows} of the {case.N} W rows, forward for all {case.M} "
+                      f"tokens through them); {tot_t:.1f} s"}
+
+
 def _oracle_sample(rows: int, qrows: int | None = None):
     """The oracle on a bounded sample of the workload: quantise + dequantise
     `qrows` rows of the 4096 x 4096 weight (all of it by default), then forward +
@@ -379,9 +529,14 @@ def main():
     ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--workload", choices=["proj7b", "smallm"], default="proj7b")
+    ap.add_argument("--n", type=int, default=8192, help="smallm: W rows (8192 or 28672)")
+    ap.add_argument("--m", type=int, default=16, help="smallm: tokens (1..64)")
     args = ap.parse_args()
     if args.impl == "reference":
         run_reference(args)
+    elif args.workload == "smallm":
+        run_smallm(args)
     else:
         run_ours(args)
 
