@@ -48,12 +48,17 @@ template <int NT_, int GROUPS_>
 struct SmallCfg {
   static constexpr int NT = NT_;          // tokens on the MMA N side (multiple of 16, <= 64)
   static constexpr int GROUPS = GROUPS_;  // dequant groups of 4 warps
-  static constexpr int KB = 2;            // 64-element K blocks per pipeline step (the MMA issuer assumes 2)
-  static constexpr int X_BYTES = NT * 128;  // one block's activation tile: NT rows x 64 bf16, 128-byte swizzle
-  static constexpr int C_BYTES = 128 * 32 * KB;  // 128 W rows x KB x 32 bytes of packed codes, 64-byte swizzle
+  static constexpr int KB = NT == 64 ? 1 : 2;  // 64-element K blocks per pipeline step
+  static constexpr int X_BYTES = NT * 128;       // one block's activation tile: NT rows x 64 bf16, 128-byte swizzle
+  static constexpr int C_ROW = 32 * KB;          // bytes of packed codes per W row and step
+  static constexpr int C_BYTES = 128 * C_ROW;    // swizzled with the C_ROW-byte TMA swizzle
   static constexpr int STAGE_BYTES = KB * X_BYTES + C_BYTES;
-  static constexpr int TSLOTS = 3;            // TMEM A slots (KB x 32 columns each)
-  static constexpr int STAGES = STAGE_BYTES <= 12288 ? 6 : 3;  // shared-memory ring, a multiple of TSLOTS
+  static constexpr int TSLOTS = 6 / KB;          // TMEM A slots (KB x 32 columns each), 192 columns in all
+  // Shared-memory ring: an even number of stages, so that with two dequant groups taking
+  // alternate steps every stage belongs to one group, and each full-barrier phase is
+  // awaited in order by a single consumer (a parity wait only tells apart the phase it
+  // waits for and the one before it).
+  static constexpr int STAGES = STAGE_BYTES <= 12288 ? 6 : 4;
   static constexpr int RING_BYTES = STAGES * STAGE_BYTES;
   static constexpr int LA_BYTES = 16384;    // Bᵀ tile: 128 W rows x 64 adapter columns, MN-major
   static constexpr int LX_BYTES = X_BYTES;  // sT tile: NT tokens x 64 adapter columns, K-major
@@ -72,11 +77,12 @@ struct SmallCfg {
   static constexpr int NUM_THREADS = 64 + DQ_THREADS;
   static_assert(NT % 16 == 0 && NT >= 16 && NT <= 64, "token tile");
   static_assert(ACC_COLS + TSLOTS * 32 * KB <= TMEM_COLS, "TMEM budget");
-  static_assert(STAGES % TSLOTS == 0, "a ring stage determines its TMEM slot");
+  static_assert(STAGES >= TSLOTS, "a slot's barrier phase is never overtaken before its waiter checks it");
   static_assert(STAGE_BYTES % 1024 == 0 && X_BYTES % 1024 == 0, "swizzle atoms stay 1024-byte aligned");
   static_assert(P_BYTES <= RING_BYTES, "the partial is parked in the drained ring");
   static_assert(2 * (SMEM_BYTES + 1024) <= 228 * 1024, "two CTAs per SM");
   static_assert(GROUPS <= TSLOTS, "each group's next slot is at most one lap ahead");
+  static_assert(STAGES % GROUPS == 0, "every ring stage belongs to one dequant group");
 };
 
 struct SmallParams {
@@ -225,7 +231,7 @@ __global__ void __launch_bounds__(C::NUM_THREADS, 2)
           mma_bf16_ts(tmem_base, a_tmem + kk * 8, bd + 2 * kk, idesc_main, acc);
           acc = 1;
         }
-        if (two) {
+        if (C::KB == 2 && two) {
 #pragma unroll
           for (int kk = 0; kk < 4; ++kk)
             mma_bf16_ts(tmem_base, a_tmem + 32 + kk * 8, bd + (C::X_BYTES >> 4) + 2 * kk, idesc_main, 1u);
@@ -319,10 +325,11 @@ __global__ void __launch_bounds__(C::NUM_THREADS, 2)
     }
     named_barrier(1, 128 * C::GROUPS);
     const float mu = *p.mean;
-    // codes tile, 64-byte rows with the 64-byte swizzle: 16-byte chunk c of row i sits at chunk
-    // c ^ ((i >> 1) & 3), so the 8 lanes of one shared-memory phase (rows i..i+7) cover all 32 banks
-    const uint32_t sw = (row >> 1) & 3;
-    const uint32_t c_row = smem_base + C::KB * C::X_BYTES + row * 64;
+    // codes tile, C_ROW-byte rows with the C_ROW-byte TMA swizzle: 16-byte chunk c of row i
+    // sits at chunk c ^ ((i >> 1) & 3) (64-byte rows) or c ^ ((i >> 2) & 1) (32-byte rows), so
+    // the 8 lanes of one shared-memory phase (rows i..i+7) cover all 32 banks
+    const uint32_t sw = C::KB == 2 ? (row >> 1) & 3 : (row >> 2) & 1;
+    const uint32_t c_row = smem_base + C::KB * C::X_BYTES + row * C::C_ROW;
     const uint32_t t_row = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + C::ACC_COLS;
     // block index of (row, block i) relative to the first staged group scale
     const int rb = static_cast<int>(static_cast<int64_t>(n0 + row) * kbt + kb_begin - (gfirst << 8));
@@ -330,7 +337,7 @@ __global__ void __launch_bounds__(C::NUM_THREADS, 2)
     for (int j = g; j < n_ss; j += C::GROUPS) {
       const int s = j % C::STAGES;
       const uint32_t ph = (j / C::STAGES) & 1;
-      const uint32_t slot = t_row + (s % C::TSLOTS) * 32 * C::KB;
+      const uint32_t slot = t_row + (j % C::TSLOTS) * 32 * C::KB;
       const int nb = n_main - j * C::KB < C::KB ? n_main - j * C::KB : C::KB;
       const bool okf = mbar_wait_bounded(&full[s], ph, abort_flag, p.dev_err, p.timeout_ns);
       if (!__all_sync(0xFFFFFFFFu, okf)) break;

@@ -250,7 +250,9 @@ static cudaError_t run_small_forward(const LaunchCtx &c, const qlora_nf4_weight 
   const int N = static_cast<int>(w.N), K = static_cast<int>(w.K);
   const int nt = static_cast<int>((M + 15) / 16) * 16;
   TmaMaps m;  // a = X, b = codes, a2 = sT, b2 = B
-  if (!map_bf16_kmajor(&m.a, X, K, M, nt) || !map_codes(&m.b, w.codes, N, K, 64, 128, 64) ||
+  const int crow = nt == 64 ? 32 : 64;  // code bytes per W row and pipeline step (SmallCfg::C_ROW)
+  static_assert(SmallCfg<64, kSmallGroups>::C_ROW == 32 && SmallCfg<48, kSmallGroups>::C_ROW == 64, "code box");
+  if (!map_bf16_kmajor(&m.a, X, K, M, nt) || !map_codes(&m.b, w.codes, N, K, crow, 128, crow) ||
       !map_bf16_kmajor(&m.a2, sT, r, M, nt) || !map_bf16_mn(&m.b2, B, N, r))
     return cudaErrorInvalidValue;
   SmallParams p;

@@ -111,10 +111,13 @@ def test_small_m_forward(m):
     (33, 512, 32768, 64),  # 48-token tile, the longest K of this path (8 splits x 64 steps)
     (64, 256, 64, 8),      # one K step, no split
     (48, 8, 128, 16),      # fewer W rows than one tile
+    (8, 40000, 64, 32),    # one K block per tile: CTAs own several whole tiles
+    (40, 12800, 256, 64),  # 48-token tile (one accumulator): ranges mix split and whole tiles
 ])
 def test_small_m_path_edges(m, n, k, r):
-    """Forward at M <= 64 (W rows on the MMA M side, tokens on N): ragged tiles,
-    K-split counts and adapter ranks; backward on the same data."""
+    """Forward at M <= 64 (W rows on the MMA M side, tokens on N, stream-K over
+    (row tile, K block) units): ragged tiles, tiles split over many CTAs or
+    owned whole, adapter ranks; backward on the same data."""
     case = inputs.LinearCase(f"smallm_edge_{m}x{n}x{k}_r{r}", M=m, N=n, K=k, r=r, alpha=16.0, w_std=0.02,
                              a_std=0.05, b_std=0.05, seed=11 + m)
     _run(case)
