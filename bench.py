@@ -58,9 +58,14 @@ TRAFFIC_CAPTURE = {"sources_sha1": "3abf9dad4be07b23c132b3cb417859c219552969",
                    "fwd_y": 46_942_976, "bwd_dx": 45_571_072}
 
 
-def kernel_sources_sha1() -> str:
+# Same for the small-M kernel (profiles/smallm_dequant_gemm_8192x8192_m16.md), per (N, M).
+SMALLM_SOURCES = ["gemm_smallm.cuh", "gemm.cuh", "nf4_decode.cuh", "ptx.cuh", "launch.cuh", "linear.cu"]
+SMALLM_TRAFFIC = {"sources_sha1": "be7e178431def2548439e796db2b1528aaaa2b5c", (8192, 16): 35_976_960}
+
+
+def kernel_sources_sha1(files=None) -> str:
     h = hashlib.sha1()
-    for f in KERNEL_SOURCES:
+    for f in files or KERNEL_SOURCES:
         with open(os.path.join(ROOT, "bit_nf4_quantised_codebook_b200", "csrc", f), "rb") as fh:
             h.update(fh.read())
     return h.hexdigest()
@@ -416,7 +421,9 @@ def run_smallm(args):
         "kernels": {"smallm_gemm_ms": round(kern_ms, 5)},
         "roofline": {"kernel": "small-M dequant GEMM", "bound": "hbm", "achieved": round(achieved, 1),
                      "peak": hbm, "unit": "GB/s", "frac": round(achieved / hbm, 4),
-                     "peak_source": f"{peak_src} HBM copy", "traffic": None,
+                     "peak_source": f"{peak_src} HBM copy",
+                     "traffic": (SMALLM_TRAFFIC.get((N, M))
+                                 if SMALLM_TRAFFIC["sources_sha1"] == kernel_sources_sha1(SMALLM_SOURCES) else None),
                      "traffic_unit": "bytes per launch (ncu dram read+write)"},
         "e2e": {"value": round(packed / (e2e_ms * 1e-3) / 1e9, 2), "unit": "GB/s",
                 "h2d_bytes_per_step": X.numel() * 2, "d2h_bytes_per_step": Y.numel() * 2, "steps": e2e_steps},
