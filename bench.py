@@ -144,6 +144,20 @@ def _dist():
     return ws, rank, local
 
 
+def max_over_ranks(x: float, device) -> float:
+    """The slowest rank's value (device time), so every rank reports the same job time."""
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([x], device=device, dtype=torch.float64)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def whole_job_rate(work_per_replica: float, world: int, seconds: float) -> float:
+    """Replicas only: every rank runs the same workload, so the job does `world` times the work."""
+    return work_per_replica * world / seconds
+
+
 def run_ours(args):
     import torch
     import torch.distributed as dist
@@ -232,14 +246,12 @@ def run_ours(args):
     fwd_ms = sum(e[0].elapsed_time(e[1]) for e in ev) / args.steps
     bwd_ms = sum(e[2].elapsed_time(e[3]) for e in ev) / args.steps
     if world > 1:
-        t = torch.tensor([ms], device=dev, dtype=torch.float64)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms = float(t.item())
+        ms = max_over_ranks(ms, dev)
     torch.cuda.synchronize()
     if int(err[0].item()) != 0:
         raise RuntimeError(f"device error word {int(err[0].item())} during timing")
     ms_step = ms / args.steps
-    value = flops * world / (ms_step * 1e-3) / 1e12
+    value = whole_job_rate(flops, world, ms_step * 1e-3) / 1e12
 
     # end to end through the public API with pinned host buffers: H2D of the step's
     # inputs (W, X, A, B, dY), the step, D2H of its results (Y, dX, dA, dB)
@@ -267,10 +279,8 @@ def run_ours(args):
     torch.cuda.synchronize()
     e2e_ms = e0.elapsed_time(e1)
     if world > 1:
-        t = torch.tensor([e2e_ms], device=dev, dtype=torch.float64)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        e2e_ms = float(t.item())
-    e2e_value = flops * world / (e2e_ms / e2e_steps * 1e-3) / 1e12
+        e2e_ms = max_over_ranks(e2e_ms, dev)
+    e2e_value = whole_job_rate(flops, world, e2e_ms / e2e_steps * 1e-3) / 1e12
 
     hbm, bf16_burst, bf16_sus, peak_src = _peaks()
     # dominant kernel: the fused dequant GEMM of the backward (dX) or forward (Y), whichever is longer
@@ -382,13 +392,11 @@ def run_smallm(args):
     ms = t0.elapsed_time(t1)
     kern_ms = sum(a.elapsed_time(b) for a, b in ev) / args.steps
     if world > 1:
-        t = torch.tensor([ms], device=dev, dtype=torch.float64)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms = float(t.item())
+        ms = max_over_ranks(ms, dev)
     if int(err[0].item()) != 0:
         raise RuntimeError(f"device error word {int(err[0].item())}")
     ms_step = ms / args.steps
-    value = packed * world / (ms_step * 1e-3) / 1e9
+    value = whole_job_rate(packed, world, ms_step * 1e-3) / 1e9
 
     # end to end: X host -> device, forward, Y device -> host
     e2e_steps = max(3, min(100, args.steps // 10))
