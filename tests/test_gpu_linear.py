@@ -150,3 +150,14 @@ def test_llama_down_projection_shape():
     case = inputs.LinearCase("down", M=512, N=4096, K=11008, r=64, alpha=16.0, w_std=0.02, a_std=0.01,
                              b_std=0.01, seed=6)
     _run(case, check_lora_alone=False)
+
+
+@pytest.mark.parametrize("n,k", [(1024, 22016), (22016, 1024)])
+def test_65b_shape_slices(n, k):
+    """Slices of the 65B shapes (W 22016 x 8192 and 8192 x 22016, 0.1% outliers)
+    cut to 2048 tokens and to 1024 W rows or 1024 columns, so that the oracle
+    stays within seconds: the long-K path (344 blocks per row) and the wide
+    grid (86 column tiles of the pair kernel)."""
+    case = inputs.LinearCase(f"65b_slice_{n}x{k}", M=2048, N=n, K=k, r=64, alpha=16.0, w_std=0.015,
+                             a_std=0.01, b_std=0.01, outlier_frac=0.001, seed=21)
+    _run(case, check_lora_alone=False)
