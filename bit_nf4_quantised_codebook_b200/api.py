@@ -23,6 +23,7 @@ EXPORTED = [
     "qlora_status_string", "qlora_build_codebook", "qlora_nf4_sizes", "qlora_workspace_size",
     "qlora_quantize", "qlora_dequantize", "qlora_linear_forward", "qlora_linear_backward",
     "qlora_kernel_launch_count", "qlora_set_timing_events", "qlora_quantize_noalloc",
+    "qlora_selftest_bounded_wait",
 ]
 
 
@@ -61,6 +62,7 @@ def lib() -> ctypes.CDLL:
         L.qlora_kernel_launch_count.argtypes = []
         L.qlora_set_timing_events.argtypes = [vp, vp, vp, vp]
         L.qlora_quantize_noalloc.argtypes = [vp, ctypes.POINTER(_Weight), vp, vp]
+        L.qlora_selftest_bounded_wait.argtypes = [ctypes.c_uint, vp, vp, vp]
         for name in EXPORTED[1:]:
             if name != "qlora_kernel_launch_count":
                 getattr(L, name).restype = i32
@@ -241,6 +243,13 @@ def qlora_set_timing_events(fwd_begin=None, fwd_end=None, bwd_begin=None, bwd_en
     h = lambda e: None if e is None else e.cuda_event
     _check(lib().qlora_set_timing_events(h(fwd_begin), h(fwd_end), h(bwd_begin), h(bwd_end)),
            "qlora_set_timing_events")
+
+
+def qlora_selftest_bounded_wait(timeout_us: int, dev_err: torch.Tensor, gave_up: torch.Tensor | None = None) -> None:
+    """Run the device self-test of the bounded-wait error path (see the C header)."""
+    _check(lib().qlora_selftest_bounded_wait(timeout_us, dev_err.data_ptr(),
+                                             None if gave_up is None else gave_up.data_ptr(), _stream()),
+           "qlora_selftest_bounded_wait")
 
 
 def bits_to_tensor(bits, device="cuda") -> torch.Tensor:

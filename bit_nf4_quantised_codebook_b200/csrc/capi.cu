@@ -347,6 +347,14 @@ qlora_status qlora_linear_backward(const qlora_nf4_weight *w, const uint16_t *X,
 
 uint64_t qlora_kernel_launch_count(void) { return g_launches.load(std::memory_order_relaxed); }
 
+qlora_status qlora_selftest_bounded_wait(unsigned timeout_us, int *dev_err, int *gave_up, void *stream) {
+  if (!dev_err || timeout_us == 0 || timeout_us > 10000000u) return QLORA_ERR_INVALID_ARG;
+  if (!device_ok()) return QLORA_ERR_NO_DEVICE;
+  cudaError_t e = launch_selftest_wait(static_cast<unsigned long long>(timeout_us) * 1000ull, dev_err, gave_up,
+                                       static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? QLORA_OK : QLORA_ERR_CUDA;
+}
+
 qlora_status qlora_set_timing_events(void *fwd_begin, void *fwd_end, void *bwd_begin, void *bwd_end) {
   g_hooks.fwd_begin = static_cast<cudaEvent_t>(fwd_begin);
   g_hooks.fwd_end = static_cast<cudaEvent_t>(fwd_end);

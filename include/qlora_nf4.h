@@ -188,13 +188,25 @@ qlora_status qlora_linear_backward(const qlora_nf4_weight *w, const uint16_t *X,
 /* ---------------------------------------------------------------- diagnostics
  * (no counterpart on the pages: instrumentation for measurement)            */
 
+/*
+ * Diagnostic with no counterpart on the pages: exercises on the device the
+ * error path that every pipeline wait of this library takes when its bound
+ * runs out.  Launches one CTA that waits, with the library's bounded mbarrier
+ * wait and a limit of timeout_us microseconds (1 .. 10^7), on a barrier that
+ * nothing arrives on.  The wait gives up, QLORA_DEVERR_TIMEOUT is OR-ed into
+ * *dev_err (required), *gave_up (device int, nullable) is set to 1, and the
+ * kernel returns normally: no fault, and the context stays usable.
+ */
+qlora_status qlora_selftest_bounded_wait(unsigned timeout_us, int *dev_err, int *gave_up, void *stream);
+
 /* Number of kernels this library has launched in this process so far. */
 uint64_t qlora_kernel_launch_count(void);
 
 /*
  * Optional timing hooks.  Each argument is a cudaEvent_t or NULL.  While set,
  * every qlora_linear_forward records fwd_begin / fwd_end on its stream
- * immediately before / after launching the fused dequant GEMM (Y), and every
+ * immediately before / after launching the dequant GEMM that produces Y (the
+ * small-M kernel when M <= 64), and every
  * qlora_linear_backward records bwd_begin / bwd_end around the fused dequant
  * GEMM that produces dX.  Passing all NULL disables the hooks.  The setting is
  * process-wide and not thread-safe.
