@@ -1,7 +1,7 @@
 """Benchmark of the QLoRA frozen-NF4 linear layer on B200.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
-                    [--workload proj7b | smallm --n N --m M]
+                    [--workload proj7b | smallm --n N --m M | adamw]
 
 One step = the whole hot path on one batch: NF4 + double quantisation of the
 bf16 weight, the forward (T = X·A, fused dequant GEMM Y = X·W_hatᵀ + sT·B) and
@@ -15,8 +15,16 @@ M = 1..64 tokens, r = 64; the weight quantised once and resident, rotated over
 enough copies to exceed L2); value = packed-weight bytes streamed per forward /
 device time (GB/s).
 
-Multi-GPU: the layer does not shard (one GPU per replica), so every rank runs
-its own replica of the workload and value sums the replicas' work over the
+--workload adamw: the fused AdamW step on the 14 adapter tensors (r = 64) of
+one LLaMA-7B decoder layer (q, k, v, o: 4096 x 4096; gate, up: 11008 x 4096;
+down: 4096 x 11008), 5.0 M parameters, float32 master values and moments plus
+the bfloat16 copies, in one launch; value = bytes moved per step / device time
+(GB/s), 30 bytes per parameter.
+
+Multi-GPU: data parallel.  Every rank runs the layer on its own 4096-token
+shard (same weight, same adapters); the adapter gradients dA and dB, one
+float32 bucket, are summed over the ranks by one NCCL all-reduce per step, as
+a data-parallel training step needs.  value sums the ranks' work over the
 slowest rank's time (weak scaling).  Rank 0 prints one JSON line.
 """
 from __future__ import annotations
@@ -187,8 +195,11 @@ def run_ours(args):
     Y = torch.empty(M, N, dtype=torch.bfloat16, device=dev)
     sT = torch.empty(M, r, dtype=torch.bfloat16, device=dev)
     dX = torch.empty(M, K, dtype=torch.bfloat16, device=dev)
-    dA = torch.empty(K, r, dtype=torch.float32, device=dev)
-    dB = torch.empty(r, N, dtype=torch.float32, device=dev)
+    # dA and dB share one float32 bucket: with several ranks (data parallel, one token
+    # shard per rank) the adapter gradients are summed by one all-reduce per step
+    gbucket = torch.empty(K * r + r * N, dtype=torch.float32, device=dev)
+    dA = gbucket[:K * r].view(K, r)
+    dB = gbucket[K * r:].view(r, N)
     ws_q = torch.empty(api.qlora_workspace_size(api.QLORA_OP_QUANTIZE, 0, N, K, 0), dtype=torch.uint8, device=dev)
     ws_f = torch.empty(api.qlora_workspace_size(api.QLORA_OP_FORWARD, M, N, K, r), dtype=torch.uint8, device=dev)
     ws_b = torch.empty(api.qlora_workspace_size(api.QLORA_OP_BACKWARD, M, N, K, r), dtype=torch.uint8, device=dev)
@@ -204,6 +215,8 @@ def run_ours(args):
         api.qlora_quantize(Wt, out=wq, ws=ws_q, dev_err=err)
         api.qlora_linear_forward(wq, Xt, At, Bt, s, Y=Y, T_save=sT, ws=ws_f, dev_err=err)
         api.qlora_linear_backward(wq, Xt, dYt, At, Bt, s, T_saved=sT, dX=dX, dA=dA, dB=dB, ws=ws_b, dev_err=err)
+        if world > 1:
+            dist.all_reduce(gbucket)  # sum of the ranks' adapter gradients (NCCL)
 
     for i in range(args.warmup):
         step(i)
@@ -299,7 +312,9 @@ def run_ours(args):
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
         "data": "synthetic (seeded numpy N(0,std) rounded to bf16)",
         "config": {"workload": WORKLOAD, "M": M, "N": N, "K": K, "r": r, "alpha": case.alpha,
-                   "global_batch": 4 * world, "seq_len": 1024, "parallelism": f"replicas x{world} (no shard)",
+                   "global_batch": 4 * world, "seq_len": 1024,
+                   "parallelism": (f"data parallel x{world}: a 4096-token shard per rank, dA/dB summed by one "
+                                   f"NCCL all-reduce per step" if world > 1 else "one GPU"),
                    "step": "quantise(W) + forward + backward",
                    "l2": f"inputs larger than L2: {NSETS} rotating input sets (W, X, dY 33.5 MB each) + 67 MB outputs"},
         "packed_weight_gbs": round(2 * packed / (ms_step * 1e-3) / 1e9, 2),
@@ -447,6 +462,137 @@ def run_smallm(args):
         dist.destroy_process_group()
 
 
+ADAMW_SHAPES = [("q", 4096, 4096), ("k", 4096, 4096), ("v", 4096, 4096), ("o", 4096, 4096),
+                ("gate", 11008, 4096), ("up", 11008, 4096), ("down", 4096, 11008)]  # (name, N out, K in)
+ADAMW_BYTES_PER_PARAM = 4 * 4 + 3 * 4 + 2  # read p, g, m, v; write p, m, v and the bfloat16 copy
+
+
+def run_adamw(args):
+    """The adapter optimiser step for one LLaMA-7B decoder layer (r = 64)."""
+    import torch
+    import torch.distributed as dist
+    from datetime import timedelta
+    from bit_nf4_quantised_codebook_b200 import api
+
+    world, rank, local = _dist()
+    torch.cuda.set_device(local)
+    if world > 1:
+        dist.init_process_group("nccl", timeout=timedelta(seconds=120), device_id=torch.device("cuda", local))
+    api.lib()
+    dev = torch.device("cuda", local)
+    r = 64
+    gen = torch.Generator(device=dev).manual_seed(0)
+    tensors, host_g, dev_g = [], [], []
+    for _, n_out, k_in in ADAMW_SHAPES:
+        for shape in ((k_in, r), (r, n_out)):  # A = L1 [K, r], B = L2 [r, N]
+            p = torch.randn(shape, generator=gen, device=dev) * 0.01
+            g = torch.randn(shape, generator=gen, device=dev)
+            tensors.append((p, torch.empty(shape, dtype=torch.bfloat16, device=dev), g,
+                            torch.zeros(shape, device=dev), torch.zeros(shape, device=dev)))
+            dev_g.append(g)
+            host_g.append(g.cpu().pin_memory())
+    nparam = sum(t[0].numel() for t in tensors)
+    step_bytes = nparam * ADAMW_BYTES_PER_PARAM
+
+    def step(i):
+        api.qlora_adamw_step(tensors, 2e-4, 0.9, 0.999, 1e-8, 0.01, i + 1)
+
+    for i in range(args.warmup):
+        step(i)
+    torch.cuda.synchronize()
+    gpu_id = None
+    try:
+        gpu_id = "GPU-" + str(torch.cuda.get_device_properties(local).uuid)
+    except Exception:
+        pass
+    sampler = ClockSampler(gpu_id)
+    sampler.start()
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    launches0 = api.qlora_kernel_launch_count()
+    sampler.mark_start()
+    t0 = torch.cuda.Event(enable_timing=True)
+    t1 = torch.cuda.Event(enable_timing=True)
+    t0.record()
+    for i in range(args.steps):
+        step(args.warmup + i)
+    t1.record()
+    torch.cuda.synchronize()
+    sampler.mark_end()
+    launches = api.qlora_kernel_launch_count() - launches0
+    clocks = sampler.stop()
+    ms = t0.elapsed_time(t1)
+    if world > 1:
+        ms = max_over_ranks(ms, dev)
+    ms_step = ms / args.steps
+    value = whole_job_rate(step_bytes, world, ms_step * 1e-3) / 1e9
+
+    # end to end: the gradients host -> device, the step, the bfloat16 parameters device -> host
+    e2e_steps = max(3, min(50, args.steps // 10))
+    host_b = [torch.empty_like(t[1], device="cpu").pin_memory() for t in tensors]
+    torch.cuda.synchronize()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for i in range(e2e_steps):
+        for hg, dg in zip(host_g, dev_g):
+            dg.copy_(hg, non_blocking=True)
+        step(args.warmup + args.steps + i)
+        for hb, t in zip(host_b, tensors):
+            hb.copy_(t[1], non_blocking=True)
+    e1.record()
+    torch.cuda.synchronize()
+    e2e_ms = e0.elapsed_time(e1) / e2e_steps
+    if world > 1:
+        e2e_ms = max_over_ranks(e2e_ms, dev)
+
+    hbm, _, _, peak_src = _peaks()
+    achieved = step_bytes / (ms_step * 1e-3) / 1e9
+    line = {
+        "metric": METRIC, "value": round(value, 2), "unit": "GB/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_step, 5),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32",
+        "data": "synthetic (seeded torch normal)",
+        "config": {"workload": "AdamW step on the r=64 adapters of one LLaMA-7B decoder layer (14 tensors)",
+                   "params": nparam, "parallelism": f"replicas x{world} (no shard)",
+                   "step": "one fused launch: decay, moments, bias-corrected update, bfloat16 copy",
+                   "l2": f"working set {step_bytes / 1e6:.0f} MB > L2"},
+        "roofline": {"kernel": "k_adamw", "bound": "hbm", "achieved": round(achieved, 1), "peak": hbm,
+                     "unit": "GB/s", "frac": round(achieved / hbm, 4), "peak_source": f"{peak_src} HBM copy",
+                     "traffic": None, "traffic_unit": "bytes per launch (ncu dram read+write)"},
+        "e2e": {"value": round(step_bytes / (e2e_ms * 1e-3) / 1e9, 2), "unit": "GB/s",
+                "h2d_bytes_per_step": nparam * 4, "d2h_bytes_per_step": nparam * 2, "steps": e2e_steps},
+        "gpu_launches": int(launches),
+        "clocks": clocks,
+    }
+    if world == 1 and rank == 0 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline_adamw()
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+def cpu_baseline_adamw(min_seconds: float = 10.0) -> dict:
+    """The oracle's AdamW step on 2^20 parameters, repeated; bytes as on the GPU."""
+    import numpy as np
+    from oracle import adamw
+    rng = np.random.default_rng(0)
+    n = 1 << 20
+    p, m, v = rng.normal(size=n) * 0.01, np.zeros(n), np.zeros(n)
+    g = rng.normal(size=n)
+    tot_t, k = 0.0, 0
+    while tot_t < min_seconds or k == 0:
+        t = time.perf_counter()
+        p, m, v = adamw.adamw_step(p, g, m, v, k + 1, 2e-4, 0.9, 0.999, 1e-8, 0.01)
+        tot_t += time.perf_counter() - t
+        k += 1
+    return {"value": round(k * n * ADAMW_BYTES_PER_PARAM / tot_t / 1e9, 4), "unit": "GB/s", "cores": os.cpu_count(),
+            "kind": "oracle", "sample": f"{k} AdamW steps on 2^20 parameters (float64 numpy); {tot_t:.1f} s"}
+
+
 def cpu_baseline_smallm(case, min_seconds: float = 10.0) -> dict:
     """The oracle on a slice of the small-M forward: quantise `rows` W rows and run
     the forward for all tokens through them; GB/s of packed weight per host second."""
@@ -544,7 +690,7 @@ def main():
     ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--workload", choices=["proj7b", "smallm"], default="proj7b")
+    ap.add_argument("--workload", choices=["proj7b", "smallm", "adamw"], default="proj7b")
     ap.add_argument("--n", type=int, default=8192, help="smallm: W rows (8192 or 28672)")
     ap.add_argument("--m", type=int, default=16, help="smallm: tokens (1..64)")
     args = ap.parse_args()
@@ -552,6 +698,8 @@ def main():
         run_reference(args)
     elif args.workload == "smallm":
         run_smallm(args)
+    elif args.workload == "adamw":
+        run_adamw(args)
     else:
         run_ours(args)
 

@@ -23,7 +23,7 @@ EXPORTED = [
     "qlora_status_string", "qlora_build_codebook", "qlora_nf4_sizes", "qlora_workspace_size",
     "qlora_quantize", "qlora_dequantize", "qlora_linear_forward", "qlora_linear_backward",
     "qlora_kernel_launch_count", "qlora_set_timing_events", "qlora_quantize_noalloc",
-    "qlora_selftest_bounded_wait",
+    "qlora_selftest_bounded_wait", "qlora_adamw_step",
 ]
 
 
@@ -34,6 +34,11 @@ class QloraError(RuntimeError):
 class _Weight(ctypes.Structure):
     _fields_ = [("N", ctypes.c_int64), ("K", ctypes.c_int64), ("codes", ctypes.c_void_p),
                 ("c2q", ctypes.c_void_p), ("c1", ctypes.c_void_p), ("mean", ctypes.c_void_p)]
+
+
+class _AdamwTensor(ctypes.Structure):
+    _fields_ = [("param", ctypes.c_void_p), ("param_bf16", ctypes.c_void_p), ("grad", ctypes.c_void_p),
+                ("m", ctypes.c_void_p), ("v", ctypes.c_void_p), ("n", ctypes.c_int64)]
 
 
 _lib = None
@@ -63,6 +68,7 @@ def lib() -> ctypes.CDLL:
         L.qlora_set_timing_events.argtypes = [vp, vp, vp, vp]
         L.qlora_quantize_noalloc.argtypes = [vp, ctypes.POINTER(_Weight), vp, vp]
         L.qlora_selftest_bounded_wait.argtypes = [ctypes.c_uint, vp, vp, vp]
+        L.qlora_adamw_step.argtypes = [ctypes.POINTER(_AdamwTensor), i32, f32, f32, f32, f32, f32, i64, vp]
         for name in EXPORTED[1:]:
             if name != "qlora_kernel_launch_count":
                 getattr(L, name).restype = i32
@@ -250,6 +256,23 @@ def qlora_selftest_bounded_wait(timeout_us: int, dev_err: torch.Tensor, gave_up:
     _check(lib().qlora_selftest_bounded_wait(timeout_us, dev_err.data_ptr(),
                                              None if gave_up is None else gave_up.data_ptr(), _stream()),
            "qlora_selftest_bounded_wait")
+
+
+def qlora_adamw_step(tensors, lr: float, beta1: float = 0.9, beta2: float = 0.999, eps: float = 1e-8,
+                     weight_decay: float = 0.0, step: int = 1) -> None:
+    """One AdamW step over up to 16 tensors in one launch.  ``tensors`` is a list of
+    (param float32, param_bf16 bfloat16 or None, grad float32, m float32, v float32)
+    CUDA tensors of equal element counts per entry; param, m, v are updated in place."""
+    arr = (_AdamwTensor * max(1, len(tensors)))()
+    for k, (p, pb, g, m, v) in enumerate(tensors):
+        n = p.numel()
+        for t, name in ((p, "param"), (g, "grad"), (m, "m"), (v, "v")):
+            _need(t, torch.float32, tuple(p.shape), name)
+        if pb is not None:
+            _need(pb, torch.bfloat16, tuple(p.shape), "param_bf16")
+        arr[k] = _AdamwTensor(p.data_ptr(), _ptr(pb), g.data_ptr(), m.data_ptr(), v.data_ptr(), n)
+    _check(lib().qlora_adamw_step(arr, len(tensors), lr, beta1, beta2, eps, weight_decay, step, _stream()),
+           "qlora_adamw_step")
 
 
 def bits_to_tensor(bits, device="cuda") -> torch.Tensor:

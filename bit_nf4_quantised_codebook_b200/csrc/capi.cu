@@ -5,6 +5,7 @@
 #include <atomic>
 #include <cstdint>
 #include <cstdlib>
+#include <cmath>
 #include <cstring>
 #include <mutex>
 #include <cuda.h>
@@ -346,6 +347,28 @@ qlora_status qlora_linear_backward(const qlora_nf4_weight *w, const uint16_t *X,
 }
 
 uint64_t qlora_kernel_launch_count(void) { return g_launches.load(std::memory_order_relaxed); }
+
+qlora_status qlora_adamw_step(const qlora_adamw_tensor *tensors, int count, float lr, float beta1, float beta2,
+                              float eps, float weight_decay, int64_t step, void *stream) {
+  if (!tensors || count < 1 || count > QLORA_ADAMW_MAX_TENSORS || step < 1) return QLORA_ERR_INVALID_ARG;
+  if (!(lr >= 0.f) || !(weight_decay >= 0.f) || !(beta1 >= 0.f && beta1 < 1.f) || !(beta2 >= 0.f && beta2 < 1.f) ||
+      !(eps > 0.f))
+    return QLORA_ERR_INVALID_ARG;
+  for (int k = 0; k < count; ++k) {
+    const qlora_adamw_tensor &t = tensors[k];
+    if (!t.param || !t.grad || !t.m || !t.v || t.n < 1) return QLORA_ERR_INVALID_ARG;
+    if (!aligned16(t.param) || !aligned16(t.grad) || !aligned16(t.m) || !aligned16(t.v) ||
+        (t.param_bf16 && !aligned16(t.param_bf16)))
+      return QLORA_ERR_MISALIGNED;
+  }
+  if (!device_ok()) return QLORA_ERR_NO_DEVICE;
+  const double bc1 = 1.0 - std::pow(static_cast<double>(beta1), static_cast<double>(step));
+  const double bc2 = 1.0 - std::pow(static_cast<double>(beta2), static_cast<double>(step));
+  if (!(bc1 > 0.0) || !(bc2 > 0.0)) return QLORA_ERR_INVALID_ARG;
+  cudaError_t e = launch_adamw(tensors, count, lr, beta1, beta2, eps, weight_decay, static_cast<double>(lr) / bc1,
+                               std::sqrt(bc2), device_sms(), static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? QLORA_OK : QLORA_ERR_CUDA;
+}
 
 qlora_status qlora_selftest_bounded_wait(unsigned timeout_us, int *dev_err, int *gave_up, void *stream) {
   if (!dev_err || timeout_us == 0 || timeout_us > 10000000u) return QLORA_ERR_INVALID_ARG;

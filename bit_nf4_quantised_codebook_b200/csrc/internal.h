@@ -29,6 +29,11 @@ cudaError_t launch_quantize(const uint16_t *W, int64_t nb, uint8_t *codes, uint8
                             int *dev_err, cudaStream_t st);
 cudaError_t launch_dequantize(const uint8_t *codes, const uint8_t *c2q, const float *c1, const float *mean,
                               int64_t nb, const Nf4Levels &lv, uint16_t *out, cudaStream_t st);
+// adamw.cu
+using AdamwTensor = qlora_adamw_tensor;
+constexpr int kAdamwMaxTensors = QLORA_ADAMW_MAX_TENSORS;
+cudaError_t launch_adamw(const AdamwTensor *t, int count, float lr, float b1, float b2, float eps, float wd,
+                         double step_size, double bc2_sqrt, int num_sms, cudaStream_t st);
 // selftest.cu
 cudaError_t launch_selftest_wait(unsigned long long timeout_ns, int *dev_err, int *gave_up, cudaStream_t st);
 

@@ -189,6 +189,37 @@ qlora_status qlora_linear_backward(const qlora_nf4_weight *w, const uint16_t *X,
  * (no counterpart on the pages: instrumentation for measurement)            */
 
 /*
+ * One AdamW step on the trained adapter factors, all tensors in one launch.
+ * "QLoRA: Efficient Finetuning of Quantized LLMs" (intuitivepapers.ai), §Where
+ * finetuning memory goes: Adam keeps a running mean and variance of each
+ * trained weight's gradients in 32-bit floats; §The QLoRA layer, end to end:
+ * only the adapters (L1 = A, L2 = B) carry gradients and optimiser state.  The
+ * update is AdamW (Loshchilov and Hutter, decoupled weight decay) in PyTorch's
+ * arrangement, per element at step t >= 1:
+ *   p <- p·(1 - lr·wd);  m <- m + (1 - b1)·(g - m);  v <- b2·v + (1 - b2)·g²;
+ *   p <- p - lr/(1 - b1^t) · m / (sqrt(v)/sqrt(1 - b2^t) + eps)
+ * in float32.  Parameters are kept as float32 master values; when param_bf16
+ * is set, the bfloat16 copy the linear layer reads (round to nearest even) is
+ * written after the update.  All pointers are device pointers, 16-byte
+ * aligned; m and v must be zero before step 1; tensors must not overlap.
+ * Errors: QLORA_ERR_INVALID_ARG for null pointers, count outside
+ * 1..QLORA_ADAMW_MAX_TENSORS, n < 1, step < 1, lr < 0, wd < 0, beta outside
+ * [0, 1) or eps <= 0; QLORA_ERR_MISALIGNED for unaligned pointers.
+ */
+#define QLORA_ADAMW_MAX_TENSORS 16
+typedef struct {
+  float *param;         /* float32 master values, updated in place */
+  uint16_t *param_bf16; /* nullable: bfloat16 copy written after the update */
+  const float *grad;    /* float32 gradient, e.g. dA or dB of qlora_linear_backward */
+  float *m;             /* first moment, float32, updated in place */
+  float *v;             /* second moment, float32, updated in place */
+  int64_t n;            /* elements */
+} qlora_adamw_tensor;
+
+qlora_status qlora_adamw_step(const qlora_adamw_tensor *tensors, int count, float lr, float beta1, float beta2,
+                              float eps, float weight_decay, int64_t step, void *stream);
+
+/*
  * Diagnostic with no counterpart on the pages: exercises on the device the
  * error path that every pipeline wait of this library takes when its bound
  * runs out.  Launches one CTA that waits, with the library's bounded mbarrier

@@ -38,3 +38,40 @@ def test_two_rank_job_time_and_rate():
         job_ms, rate = out[r]
         assert job_ms == pytest.approx(15.0)                   # max over ranks, on every rank
         assert rate == pytest.approx(2.0 * world / 15e-3)      # replicas' work / slowest time
+
+
+def _dp_rank(rank: int, world: int, port: int, out):
+    """Each rank: the oracle's adapter gradients on its token shard, then the same
+    sum-all-reduce bench.py applies to its dA/dB bucket."""
+    import numpy as np
+    from bit_nf4_quantised_codebook_b200 import inputs
+    from oracle import linear, nf4
+
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port), RANK=str(rank), WORLD_SIZE=str(world))
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    try:
+        case = inputs.LinearCase("dp", M=64, N=128, K=192, r=16, alpha=16.0, w_std=0.02, a_std=0.05,
+                                 b_std=0.05, seed=9)
+        what = nf4.dequantize_nf4(nf4.quantize_nf4(case.W()))
+        X, dY = case.X(), case.dY()
+        sl = slice(rank * case.M // world, (rank + 1) * case.M // world)  # this rank's token shard
+        g = linear.backward(X[sl], dY[sl], what, case.A(), case.B(), case.s)
+        bucket = torch.tensor(np.concatenate([g["dA"].ravel(), g["dB"].ravel()]))
+        dist.all_reduce(bucket)
+        full = linear.backward(X, dY, what, case.A(), case.B(), case.s)
+        out[rank] = (bucket.numpy(), np.concatenate([full["dA"].ravel(), full["dB"].ravel()]))
+        dist.barrier()
+    finally:
+        dist.destroy_process_group()
+
+
+def test_data_parallel_adapter_gradients_sum_over_shards():
+    """The exchange step of the data-parallel bench: summing the shards' dA/dB gives
+    the whole batch's gradients (they are sums over tokens)."""
+    world = 2
+    out = mp.Manager().dict()
+    mp.spawn(_dp_rank, args=(world, _free_port(), out), nprocs=world, join=True)
+    for r in range(world):
+        got, full = out[r]
+        assert got.shape == full.shape
+        assert abs(got - full).max() <= 1e-12 * max(1.0, abs(full).max())

@@ -88,3 +88,25 @@ def test_product_path_has_no_cpu_fallback():
         if f.endswith(".py"):
             txt = open(os.path.join(pkg, f)).read()
             assert "import oracle" not in txt and "from oracle" not in txt, f
+
+
+def test_adamw_validation(api):
+    """qlora_adamw_step rejects bad arguments before any launch (1 = invalid argument,
+    3 = misaligned pointer)."""
+    L = api.lib()
+    T = api._AdamwTensor
+    good = (T * 1)(T(16, 0, 32, 48, 64, 8))  # 16-byte aligned (fake) addresses; never dereferenced
+    args = (0.001, 0.9, 0.999, 1e-8, 0.0)
+    assert L.qlora_adamw_step(None, 1, *args, 1, None) == 1
+    assert L.qlora_adamw_step(good, 0, *args, 1, None) == 1
+    assert L.qlora_adamw_step(good, 17, *args, 1, None) == 1
+    assert L.qlora_adamw_step(good, 1, *args, 0, None) == 1           # step < 1
+    assert L.qlora_adamw_step(good, 1, 0.001, 1.0, 0.999, 1e-8, 0.0, 1, None) == 1
+    assert L.qlora_adamw_step(good, 1, 0.001, 0.9, 0.999, 0.0, 0.0, 1, None) == 1
+    assert L.qlora_adamw_step(good, 1, -1.0, 0.9, 0.999, 1e-8, 0.0, 1, None) == 1
+    nul = (T * 1)(T(16, 0, 0, 48, 64, 8))
+    assert L.qlora_adamw_step(nul, 1, *args, 1, None) == 1
+    empty = (T * 1)(T(16, 0, 32, 48, 64, 0))
+    assert L.qlora_adamw_step(empty, 1, *args, 1, None) == 1
+    mis = (T * 1)(T(20, 0, 32, 48, 64, 8))
+    assert L.qlora_adamw_step(mis, 1, *args, 1, None) == 3
