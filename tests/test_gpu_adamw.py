@@ -27,8 +27,10 @@ def test_adamw_matches_oracle():
     Mm = [torch.zeros(x.shape, dtype=torch.float32, device=dev) for x in p0]
     Vv = [torch.zeros(x.shape, dtype=torch.float32, device=dev) for x in p0]
     ref = [(x.astype(np.float64), np.zeros(x.shape), np.zeros(x.shape)) for x in p0]
+    gmax = np.zeros(len(shapes))  # largest |gradient| seen per tensor
     for t in range(1, 4):
         grads = [(rng.normal(size=s) * 10.0 ** rng.integers(-3, 1)).astype(np.float32) for s in shapes]
+        gmax = np.maximum(gmax, [np.abs(g).max() for g in grads])
         G = [torch.tensor(g, device=dev) for g in grads]
         a.qlora_adamw_step(list(zip(P, Pb, G, Mm, Vv)), LR, B1, B2, EPS, WD, t)
         ref = [adamw.adamw_step(p, g.astype(np.float64), m, v, t, LR, B1, B2, EPS, WD)
@@ -39,8 +41,10 @@ def test_adamw_matches_oracle():
         p_g = P[k].cpu().numpy().astype(np.float64)
         m_g = Mm[k].cpu().numpy().astype(np.float64)
         v_g = Vv[k].cpu().numpy().astype(np.float64)
-        np.testing.assert_allclose(m_g, m_ref, rtol=1e-5, atol=1e-12)
-        np.testing.assert_allclose(v_g, v_ref, rtol=1e-5, atol=1e-18)
+        # float32 moments: each step rounds m + (1-b1)(g-m) and b2 v + (1-b2) g^2, an error of a
+        # few float32 ulps of the gradient scale; m can cancel to near zero, so the bound is absolute
+        np.testing.assert_allclose(m_g, m_ref, rtol=1e-5, atol=3 * 2.0 ** -23 * gmax[k])
+        np.testing.assert_allclose(v_g, v_ref, rtol=1e-5, atol=3 * 2.0 ** -23 * gmax[k] ** 2)
         # float32 parameters: rounding of p (|p| ~ 0.01) and of three steps of size ~lr
         assert np.max(np.abs(p_g - p_ref)) <= 1e-8
         pb = Pb[k].cpu().view(torch.int16).numpy().view(np.uint16)
