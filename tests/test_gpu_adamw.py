@@ -45,8 +45,10 @@ def test_adamw_matches_oracle():
         # few float32 ulps of the gradient scale; m can cancel to near zero, so the bound is absolute
         np.testing.assert_allclose(m_g, m_ref, rtol=1e-5, atol=3 * 2.0 ** -23 * gmax[k])
         np.testing.assert_allclose(v_g, v_ref, rtol=1e-5, atol=3 * 2.0 ** -23 * gmax[k] ** 2)
-        # float32 parameters: rounding of p (|p| ~ 0.01) and of three steps of size ~lr
-        assert np.max(np.abs(p_g - p_ref)) <= 1e-8
+        # float32 parameters: two roundings of p per step (decay, update) over three steps, a
+        # few float32 ulps of the largest |p|, plus the float32 error of the steps themselves
+        tol = 8 * 2.0 ** -24 * np.abs(p_ref).max() + 3 * LR * 1e-5
+        assert np.max(np.abs(p_g - p_ref)) <= tol
         pb = Pb[k].cpu().view(torch.int16).numpy().view(np.uint16)
         assert np.array_equal(pb, f32_to_bf16_rne(P[k].cpu().numpy()))   # the copy is RN(param)
         ulp = np.abs(bf16_to_f64(f32_to_bf16_rne(p_ref.astype(np.float32))) - bf16_to_f64(pb))
