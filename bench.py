@@ -493,9 +493,10 @@ def run_adamw(args):
             host_g.append(g.cpu().pin_memory())
     nparam = sum(t[0].numel() for t in tensors)
     step_bytes = nparam * ADAMW_BYTES_PER_PARAM
+    group = api.AdamwGroup(tensors)  # marshalled once; each step is the C call alone
 
     def step(i):
-        api.qlora_adamw_step(tensors, 2e-4, 0.9, 0.999, 1e-8, 0.01, i + 1)
+        group.step(2e-4, 0.9, 0.999, 1e-8, 0.01, i + 1)
 
     for i in range(args.warmup):
         step(i)

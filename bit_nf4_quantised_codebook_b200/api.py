@@ -258,21 +258,35 @@ def qlora_selftest_bounded_wait(timeout_us: int, dev_err: torch.Tensor, gave_up:
            "qlora_selftest_bounded_wait")
 
 
+class AdamwGroup:
+    """Up to 16 adapter tensors prepared once for qlora_adamw_step: the tensors are
+    checked and the descriptor array is built here, so that each step() is only
+    the C call.  ``tensors`` is a list of (param float32, param_bf16 bfloat16 or
+    None, grad float32, m float32, v float32) CUDA tensors; the caller keeps
+    them alive and in place (param, m, v are updated in place)."""
+
+    def __init__(self, tensors):
+        self.count = len(tensors)
+        self.arr = (_AdamwTensor * max(1, self.count))()
+        self.keep = list(tensors)
+        for k, (p, pb, g, m, v) in enumerate(tensors):
+            for t, name in ((p, "param"), (g, "grad"), (m, "m"), (v, "v")):
+                _need(t, torch.float32, tuple(p.shape), name)
+            if pb is not None:
+                _need(pb, torch.bfloat16, tuple(p.shape), "param_bf16")
+            self.arr[k] = _AdamwTensor(p.data_ptr(), _ptr(pb), g.data_ptr(), m.data_ptr(), v.data_ptr(), p.numel())
+
+    def step(self, lr: float, beta1: float = 0.9, beta2: float = 0.999, eps: float = 1e-8,
+             weight_decay: float = 0.0, step: int = 1) -> None:
+        _check(lib().qlora_adamw_step(self.arr, self.count, lr, beta1, beta2, eps, weight_decay, step, _stream()),
+               "qlora_adamw_step")
+
+
 def qlora_adamw_step(tensors, lr: float, beta1: float = 0.9, beta2: float = 0.999, eps: float = 1e-8,
                      weight_decay: float = 0.0, step: int = 1) -> None:
-    """One AdamW step over up to 16 tensors in one launch.  ``tensors`` is a list of
-    (param float32, param_bf16 bfloat16 or None, grad float32, m float32, v float32)
-    CUDA tensors of equal element counts per entry; param, m, v are updated in place."""
-    arr = (_AdamwTensor * max(1, len(tensors)))()
-    for k, (p, pb, g, m, v) in enumerate(tensors):
-        n = p.numel()
-        for t, name in ((p, "param"), (g, "grad"), (m, "m"), (v, "v")):
-            _need(t, torch.float32, tuple(p.shape), name)
-        if pb is not None:
-            _need(pb, torch.bfloat16, tuple(p.shape), "param_bf16")
-        arr[k] = _AdamwTensor(p.data_ptr(), _ptr(pb), g.data_ptr(), m.data_ptr(), v.data_ptr(), n)
-    _check(lib().qlora_adamw_step(arr, len(tensors), lr, beta1, beta2, eps, weight_decay, step, _stream()),
-           "qlora_adamw_step")
+    """One AdamW step over up to 16 tensors in one launch (see AdamwGroup for the
+    tensor list); for repeated steps on the same tensors, keep an AdamwGroup."""
+    AdamwGroup(tensors).step(lr, beta1, beta2, eps, weight_decay, step)
 
 
 def bits_to_tensor(bits, device="cuda") -> torch.Tensor:
