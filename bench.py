@@ -71,6 +71,11 @@ SMALLM_SOURCES = ["gemm_smallm.cuh", "gemm.cuh", "nf4_decode.cuh", "ptx.cuh", "l
 SMALLM_TRAFFIC = {"sources_sha1": "be7e178431def2548439e796db2b1528aaaa2b5c", (8192, 16): 35_976_960}
 
 
+# Same for the AdamW kernel (profiles/adamw_llama7b_layer_adapters.md).
+ADAMW_SOURCES = ["adamw.cu", "ptx.cuh", "launch.cuh"]
+ADAMW_TRAFFIC = {"sources_sha1": "0064428f763192ff27c64743df1b67afd4a73e71", "bytes": 90_732_000}
+
+
 def kernel_sources_sha1(files=None) -> str:
     h = hashlib.sha1()
     for f in files or KERNEL_SOURCES:
@@ -561,7 +566,9 @@ def run_adamw(args):
                    "l2": f"working set {step_bytes / 1e6:.0f} MB > L2"},
         "roofline": {"kernel": "k_adamw", "bound": "hbm", "achieved": round(achieved, 1), "peak": hbm,
                      "unit": "GB/s", "frac": round(achieved / hbm, 4), "peak_source": f"{peak_src} HBM copy",
-                     "traffic": None, "traffic_unit": "bytes per launch (ncu dram read+write)"},
+                     "traffic": (ADAMW_TRAFFIC["bytes"] if ADAMW_TRAFFIC["sources_sha1"] ==
+                                 kernel_sources_sha1(ADAMW_SOURCES) else None),
+                     "traffic_unit": "bytes per launch (ncu dram read+write)"},
         "e2e": {"value": round(step_bytes / (e2e_ms * 1e-3) / 1e9, 2), "unit": "GB/s",
                 "h2d_bytes_per_step": nparam * 4, "d2h_bytes_per_step": nparam * 2, "steps": e2e_steps},
         "gpu_launches": int(launches),
