@@ -42,6 +42,16 @@ def normal_bf16(shape, std: float, seed: int) -> np.ndarray:
     return to_bf16_bits(rng.standard_normal(size=shape) * std)
 
 
+def dyadic_bf16(shape, k_max: int, exp2: int, seed: int) -> np.ndarray:
+    """Integers drawn uniformly from [-k_max, k_max], times 2^-exp2.  Exact in
+    bfloat16 for k_max <= 256.  With small k_max every product of two such
+    values, and every sum of a few hundred of them, is exact in float32, so a
+    contraction over them has one correct result whatever its summation order."""
+    rng = np.random.default_rng(seed)
+    v = rng.integers(-k_max, k_max + 1, size=shape).astype(np.float64) * 2.0 ** -exp2
+    return to_bf16_bits(v)
+
+
 def weight_bf16(n: int, k: int, std: float, seed: int, outlier_frac: float = 0.0) -> np.ndarray:
     rng = np.random.default_rng(seed)
     w = rng.standard_normal(size=(n, k)) * std
