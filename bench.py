@@ -583,6 +583,186 @@ def run_adamw(args):
         dist.destroy_process_group()
 
 
+MERGE_SHAPES = ADAMW_SHAPES  # the seven linears of one LLaMA-7B decoder layer
+
+
+def merge_bytes(N: int, K: int, r: int) -> int:
+    """Algorithmic bytes of one merge: the stored weight read and written once
+    (codes, E4M3 constants, group scales, mean) and the adapter read once."""
+    nb = N * K // 64
+    packed = N * K // 2 + nb + 4 * (-(-nb // 256)) + 4
+    return 2 * packed + 2 * r * (K + N)
+
+
+def merge_kernel_bytes(N: int, K: int, r: int) -> int:
+    """Algorithmic bytes of the merge-and-code kernel: old codes and constants
+    in, the adapter in, new codes and the float32 block absmax out."""
+    nb = N * K // 64
+    return N * K // 2 + nb + 4 * (-(-nb // 256)) + 4 + 2 * r * (K + N) + N * K // 2 + 4 * nb
+
+
+def run_merge(args):
+    """Merge the r = 64 adapters of one LLaMA-7B layer into its NF4 weights and
+    requantise them: a step is the seven merges."""
+    import torch
+    import torch.distributed as dist
+    from datetime import timedelta
+    from bit_nf4_quantised_codebook_b200 import api, inputs
+
+    world, rank, local = _dist()
+    torch.cuda.set_device(local)
+    if world > 1:
+        dist.init_process_group("nccl", timeout=timedelta(seconds=120), device_id=torch.device("cuda", local))
+    api.lib()
+    dev = torch.device("cuda", local)
+    r, alpha = 64, 16.0
+    s = alpha / r
+    ncopy = 2  # two resident copies of the layer (each > 200 MB read + written per step) in rotation
+    mats, adapters, outs = [], [], []
+    for j, (_, N, K) in enumerate(MERGE_SHAPES):
+        W = api.bits_to_tensor(inputs.weight_bf16(N, K, 0.02, 10 * j, 0.001), dev)
+        mats.append([api.qlora_quantize(W) for _ in range(ncopy)])
+        outs.append([api.alloc_weight(N, K, dev) for _ in range(ncopy)])
+        del W
+        adapters.append((api.bits_to_tensor(inputs.normal_bf16((K, r), 0.01, 10 * j + 2), dev),
+                         api.bits_to_tensor(inputs.normal_bf16((r, N), 0.01, 10 * j + 3), dev)))
+    ws = torch.empty(max(api.qlora_workspace_size(api.QLORA_OP_MERGE, 0, N, K, r) for _, N, K in MERGE_SHAPES),
+                     dtype=torch.uint8, device=dev)
+    err = api.new_error_word(dev)
+    step_bytes = sum(merge_bytes(N, K, r) for _, N, K in MERGE_SHAPES)
+    kern_bytes = sum(merge_kernel_bytes(N, K, r) for _, N, K in MERGE_SHAPES)
+
+    def step(i, hooks=None):
+        c = i % ncopy
+        for j in range(len(MERGE_SHAPES)):
+            if hooks is not None:
+                api.qlora_set_timing_events(hooks[j][0], hooks[j][1])
+            A, B = adapters[j]
+            api.qlora_merge_requantize(mats[j][c], A, B, s, out=outs[j][c], ws=ws, dev_err=err)
+
+    for i in range(args.warmup):
+        step(i)
+    torch.cuda.synchronize()
+    nj = len(MERGE_SHAPES)
+    ev = [[[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(nj)] for _ in range(args.steps)]
+    gpu_id = None
+    try:
+        gpu_id = "GPU-" + str(torch.cuda.get_device_properties(local).uuid)
+    except Exception:
+        pass
+    sampler = ClockSampler(gpu_id)
+    sampler.start()
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    launches0 = api.qlora_kernel_launch_count()
+    sampler.mark_start()
+    t0 = torch.cuda.Event(enable_timing=True)
+    t1 = torch.cuda.Event(enable_timing=True)
+    t0.record()
+    for i in range(args.steps):
+        step(i)
+    t1.record()
+    torch.cuda.synchronize()
+    sampler.mark_end()
+    launches = api.qlora_kernel_launch_count() - launches0
+    # the merge-and-code kernels alone, events around each (a separate loop: the
+    # events end the programmatic overlap between the kernels of a merge)
+    for i in range(args.steps):
+        step(i, ev[i])
+    torch.cuda.synchronize()
+    api.qlora_set_timing_events()
+    clocks = sampler.stop()
+    ms = t0.elapsed_time(t1)
+    kern_ms = sum(a.elapsed_time(b) for row in ev for a, b in row) / args.steps
+    if world > 1:
+        ms = max_over_ranks(ms, dev)
+    if int(err[0].item()) != 0:
+        raise RuntimeError(f"device error word {int(err[0].item())}")
+    ms_step = ms / args.steps
+    value = whole_job_rate(step_bytes, world, ms_step * 1e-3) / 1e9
+
+    # end to end: each weight's stored form and its adapter host -> device, merge,
+    # the new stored form device -> host
+    e2e_steps = max(3, min(20, args.steps // 10))
+    host_in, host_out, h2d, d2h = [], [], 0, 0
+    for j in range(nj):
+        q, o = mats[j][0], outs[j][0]
+        A, B = adapters[j]
+        host_in.append([t.cpu().pin_memory() for t in (q.codes, q.c2q, q.c1, q.mean, A, B)])
+        host_out.append([torch.empty_like(t, device="cpu").pin_memory() for t in (o.codes, o.c2q, o.c1, o.mean)])
+        h2d += sum(t.numel() * t.element_size() for t in host_in[-1])
+        d2h += sum(t.numel() * t.element_size() for t in host_out[-1])
+    torch.cuda.synchronize()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(e2e_steps):
+        for j in range(nj):
+            q, o = mats[j][0], outs[j][0]
+            A, B = adapters[j]
+            for dst, src in zip((q.codes, q.c2q, q.c1, q.mean, A, B), host_in[j]):
+                dst.copy_(src, non_blocking=True)
+            api.qlora_merge_requantize(q, A, B, s, out=o, ws=ws, dev_err=err)
+            for dst, src in zip(host_out[j], (o.codes, o.c2q, o.c1, o.mean)):
+                dst.copy_(src, non_blocking=True)
+    e1.record()
+    torch.cuda.synchronize()
+    e2e_ms = e0.elapsed_time(e1) / e2e_steps
+
+    hbm, _, _, peak_src = _peaks()
+    achieved = kern_bytes / (kern_ms * 1e-3) / 1e9
+    line = {
+        "metric": "merge + requantise throughput (stored weight read and written, adapter read)",
+        "value": round(value, 2), "unit": "GB/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_step, 5),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32",
+        "data": "synthetic (seeded numpy N(0,std) rounded to bf16; W with 0.1% t(3) outliers)",
+        "config": {"workload": f"adapter merge + NF4 requantisation of one LLaMA-7B layer's 7 linears, "
+                               f"LoRA r={r} alpha={alpha}",
+                   "shapes": [f"{nm} {N}x{K}" for nm, N, K in MERGE_SHAPES], "r": r,
+                   "parallelism": f"replicas x{world} (no shard)",
+                   "step": "7 x qlora_merge_requantize (merge-and-code kernel, group sums, mean, E4M3 codes)",
+                   "l2": f"{ncopy} copies of the layer in rotation; each step reads and writes "
+                         f"{step_bytes / 1e6:.0f} MB (> L2)"},
+        "kernels": {"merge_kernel_ms_per_step": round(kern_ms, 5)},
+        "roofline": {"kernel": "k_merge_quant", "bound": "hbm", "achieved": round(achieved, 1), "peak": hbm,
+                     "unit": "GB/s", "frac": round(achieved / hbm, 4), "peak_source": f"{peak_src} HBM copy",
+                     "traffic": None, "traffic_unit": "bytes per launch (ncu dram read+write)"},
+        "e2e": {"value": round(step_bytes / (e2e_ms * 1e-3) / 1e9, 2), "unit": "GB/s",
+                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": e2e_steps},
+        "gpu_launches": int(launches),
+        "clocks": clocks,
+    }
+    if world == 1 and rank == 0 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline_merge()
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+def cpu_baseline_merge(min_seconds: float = 10.0) -> dict:
+    """The oracle's merge + requantisation on a 256-row slice of the 4096 x 4096
+    q projection, repeated; GB/s counted as on the GPU."""
+    from bit_nf4_quantised_codebook_b200 import inputs
+    from oracle import merge, nf4
+    rows, K, r = 256, 4096, 64
+    q = nf4.quantize_nf4(inputs.weight_bf16(4096, K, 0.02, 0, 0.001)[:rows])
+    A = inputs.normal_bf16((K, r), 0.01, 2)
+    B = inputs.normal_bf16((r, 4096), 0.01, 3)[:, :rows]
+    tot_t, n = 0.0, 0
+    while tot_t < min_seconds or n == 0:
+        t = time.perf_counter()
+        merge.merge_requantize(q, A, B, 0.25)
+        tot_t += time.perf_counter() - t
+        n += 1
+    return {"value": round(n * merge_bytes(rows, K, r) / tot_t / 1e9, 6), "unit": "GB/s", "cores": os.cpu_count(),
+            "kind": "oracle", "sample": f"{n} x merge + requantise of {rows} of the 4096 rows of the 4096x4096 "
+                                        f"q projection (float64 numpy); {tot_t:.1f} s"}
+
+
 def cpu_baseline_adamw(min_seconds: float = 10.0) -> dict:
     """The oracle's AdamW step on 2^20 parameters, repeated; bytes as on the GPU."""
     import numpy as np
@@ -698,7 +878,7 @@ def main():
     ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--workload", choices=["proj7b", "smallm", "adamw"], default="proj7b")
+    ap.add_argument("--workload", choices=["proj7b", "smallm", "adamw", "merge"], default="proj7b")
     ap.add_argument("--n", type=int, default=8192, help="smallm: W rows (8192 or 28672)")
     ap.add_argument("--m", type=int, default=16, help="smallm: tokens (1..64)")
     args = ap.parse_args()
@@ -708,6 +888,8 @@ def main():
         run_smallm(args)
     elif args.workload == "adamw":
         run_adamw(args)
+    elif args.workload == "merge":
+        run_merge(args)
     else:
         run_ours(args)
 

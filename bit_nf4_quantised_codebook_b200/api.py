@@ -16,14 +16,14 @@ import torch
 _PKG = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_PKG, "libqlora_nf4.so")
 
-QLORA_OP_QUANTIZE, QLORA_OP_FORWARD, QLORA_OP_BACKWARD = 0, 1, 2
+QLORA_OP_QUANTIZE, QLORA_OP_FORWARD, QLORA_OP_BACKWARD, QLORA_OP_MERGE = 0, 1, 2, 3
 QLORA_DEVERR_NONFINITE, QLORA_DEVERR_TIMEOUT = 1, 2
 
 EXPORTED = [
     "qlora_status_string", "qlora_build_codebook", "qlora_nf4_sizes", "qlora_workspace_size",
     "qlora_quantize", "qlora_dequantize", "qlora_linear_forward", "qlora_linear_backward",
     "qlora_kernel_launch_count", "qlora_set_timing_events", "qlora_quantize_noalloc",
-    "qlora_selftest_bounded_wait", "qlora_adamw_step",
+    "qlora_selftest_bounded_wait", "qlora_adamw_step", "qlora_merge_requantize",
 ]
 
 
@@ -69,6 +69,8 @@ def lib() -> ctypes.CDLL:
         L.qlora_quantize_noalloc.argtypes = [vp, ctypes.POINTER(_Weight), vp, vp]
         L.qlora_selftest_bounded_wait.argtypes = [ctypes.c_uint, vp, vp, vp]
         L.qlora_adamw_step.argtypes = [ctypes.POINTER(_AdamwTensor), i32, f32, f32, f32, f32, f32, i64, vp]
+        L.qlora_merge_requantize.argtypes = [ctypes.POINTER(_Weight), vp, vp, i32, f32, ctypes.POINTER(_Weight),
+                                             vp, vp, sz, vp, vp]
         for name in EXPORTED[1:]:
             if name != "qlora_kernel_launch_count":
                 getattr(L, name).restype = i32
@@ -186,6 +188,26 @@ def qlora_dequantize(w: NF4Weight, out: torch.Tensor | None = None) -> torch.Ten
     _need(out, torch.bfloat16, (w.N, w.K), "W_out")
     s = w.c_struct()
     _check(lib().qlora_dequantize(ctypes.byref(s), out.data_ptr(), _stream()), "qlora_dequantize")
+    return out
+
+
+def qlora_merge_requantize(w: NF4Weight, A: torch.Tensor, B: torch.Tensor, s: float, out: NF4Weight | None = None,
+                           W_merged: torch.Tensor | None = None, ws: torch.Tensor | None = None,
+                           dev_err: torch.Tensor | None = None) -> NF4Weight:
+    """W_eff = bf16(float32(W_hat + s·(A·B)ᵀ)) requantised into ``out`` (a new
+    weight by default; ``out=w`` merges in place).  ``W_merged`` (N x K bf16)
+    optionally receives W_eff."""
+    r = A.shape[1]
+    _need(A, torch.bfloat16, (w.K, r), "A")
+    _need(B, torch.bfloat16, (r, w.N), "B")
+    if W_merged is not None:
+        _need(W_merged, torch.bfloat16, (w.N, w.K), "W_merged")
+    out = out or alloc_weight(w.N, w.K, A.device)
+    ws = _workspace(QLORA_OP_MERGE, 0, w.N, w.K, r, ws, A.device)
+    sw, so = w.c_struct(), out.c_struct()
+    _check(lib().qlora_merge_requantize(ctypes.byref(sw), A.data_ptr(), B.data_ptr(), r, s, ctypes.byref(so),
+                                        _ptr(W_merged), ws.data_ptr(), ws.numel(), _ptr(dev_err), _stream()),
+           "qlora_merge_requantize")
     return out
 
 

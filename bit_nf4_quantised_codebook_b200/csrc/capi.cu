@@ -163,7 +163,7 @@ LinearPlan make_plan(int op, int64_t M, int64_t N, int64_t K, int r, int num_sms
     off = align256(off + bytes);
     return o;
   };
-  if (op == QLORA_OP_QUANTIZE) {
+  if (op == QLORA_OP_QUANTIZE || op == QLORA_OP_MERGE) {
     const int64_t nb = N * K / 64;
     const int64_t ng = (nb + 255) / 256;
     int64_t size = 1;
@@ -255,11 +255,11 @@ qlora_status qlora_nf4_sizes(int64_t N, int64_t K, size_t *codes_bytes, size_t *
 qlora_status qlora_workspace_size(int op, int64_t M, int64_t N, int64_t K, int r, size_t *bytes) {
   if (!bytes || N < 1 || K < 64) return QLORA_ERR_INVALID_ARG;
   if (K % 64 != 0) return QLORA_ERR_UNSUPPORTED_SHAPE;
-  if (op != QLORA_OP_QUANTIZE) {
+  if (op < QLORA_OP_QUANTIZE || op > QLORA_OP_MERGE) return QLORA_ERR_INVALID_ARG;
+  if (op == QLORA_OP_FORWARD || op == QLORA_OP_BACKWARD) {
     if (M < 1 || r < 1) return QLORA_ERR_INVALID_ARG;
     if (r % 8 != 0 || r > 256) return QLORA_ERR_UNSUPPORTED_SHAPE;
   }
-  if (op < QLORA_OP_QUANTIZE || op > QLORA_OP_BACKWARD) return QLORA_ERR_INVALID_ARG;
   *bytes = make_plan(op, M, N, K, r, device_sms()).bytes;
   return QLORA_OK;
 }
@@ -297,6 +297,52 @@ qlora_status qlora_dequantize(const qlora_nf4_weight *w, uint16_t *W_out, void *
   std::memcpy(lv.q, g.levels, sizeof(lv.q));
   cudaError_t e = launch_dequantize(w->codes, w->c2q, w->c1, w->mean, w->N * w->K / 64, lv, W_out,
                                     static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? QLORA_OK : QLORA_ERR_CUDA;
+}
+
+// True when [a, a+na) and [b, b+nb) share a byte.
+static bool overlap(const void *a, size_t na, const void *b, size_t nb) {
+  const uintptr_t x = reinterpret_cast<uintptr_t>(a), y = reinterpret_cast<uintptr_t>(b);
+  return x < y + nb && y < x + na;
+}
+
+qlora_status qlora_merge_requantize(const qlora_nf4_weight *w, const uint16_t *A, const uint16_t *B, int r, float s,
+                                    const qlora_nf4_weight *out, uint16_t *W_merged, void *ws, size_t ws_bytes,
+                                    int *dev_err, void *stream) {
+  qlora_status st = check_weight(w);
+  if (st != QLORA_OK) return st;
+  if ((st = check_weight(out)) != QLORA_OK) return st;
+  if (!A || !B || out->N != w->N || out->K != w->K || r < 1) return QLORA_ERR_INVALID_ARG;
+  if (r % 8 != 0 || r > 256 || w->N % 8 != 0) return QLORA_ERR_UNSUPPORTED_SHAPE;
+  if (!aligned16(A) || !aligned16(B) || (W_merged && !aligned16(W_merged))) return QLORA_ERR_MISALIGNED;
+  const int64_t nb = w->N * w->K / 64;
+  const size_t in_sz[4] = {static_cast<size_t>(w->N * w->K / 2), static_cast<size_t>(nb),
+                           static_cast<size_t>((nb + 255) / 256) * 4, 4};
+  const void *in_p[4] = {w->codes, w->c2q, w->c1, w->mean};
+  const void *out_p[4] = {out->codes, out->c2q, out->c1, out->mean};
+  for (int i = 0; i < 4; ++i)
+    for (int j = 0; j < 4; ++j)
+      if (!(i == j && in_p[i] == out_p[j]) && overlap(in_p[i], in_sz[i], out_p[j], in_sz[j]))
+        return QLORA_ERR_INVALID_ARG;
+  if (W_merged)
+    for (int i = 0; i < 4; ++i)
+      if (overlap(W_merged, static_cast<size_t>(w->N * w->K) * 2, in_p[i], in_sz[i]) ||
+          overlap(W_merged, static_cast<size_t>(w->N * w->K) * 2, out_p[i], in_sz[i]))
+        return QLORA_ERR_INVALID_ARG;
+  if (!device_ok()) return QLORA_ERR_NO_DEVICE;
+  const LinearPlan pl = make_plan(QLORA_OP_MERGE, 0, w->N, w->K, r, device_sms());
+  if (!ws || ws_bytes < pl.bytes) return QLORA_ERR_WORKSPACE;
+  if (!aligned16(ws)) return QLORA_ERR_MISALIGNED;
+  Globals &g = globals();
+  Nf4Levels lv;
+  std::memcpy(lv.q, g.levels, sizeof(lv.q));
+  Nf4Thresholds thr;
+  std::memcpy(thr.t, g.thresholds, sizeof(thr.t));
+  uint8_t *w8 = static_cast<uint8_t *>(ws);
+  const cudaError_t e = launch_merge_requantize(*w, A, B, r, s, *out, W_merged,
+                                                reinterpret_cast<float *>(w8 + pl.off_absmax),
+                                                reinterpret_cast<double *>(w8 + pl.off_gsum), pl.gsum_size, lv, thr,
+                                                dev_err, g.timeout_ns, static_cast<cudaStream_t>(stream));
   return e == cudaSuccess ? QLORA_OK : QLORA_ERR_CUDA;
 }
 

@@ -27,8 +27,21 @@ void build_codebook_f32(float levels[16], float thresholds[15]);
 cudaError_t launch_quantize(const uint16_t *W, int64_t nb, uint8_t *codes, uint8_t *c2q, float *c1, float *mean,
                             float *ws_absmax, double *ws_gsum, int64_t gsum_size, const Nf4Thresholds &thr,
                             int *dev_err, cudaStream_t st);
+// The second quantisation from block constants already in ws_absmax: group
+// sums (launch_group_sums, when the caller has not formed them), the fixed-order
+// mean, then the E4M3 codes and group scales.
+cudaError_t launch_group_sums(const float *ws_absmax, int64_t nb, double *ws_gsum, cudaStream_t st);
+cudaError_t launch_mean_and_double_quant(const float *ws_absmax, int64_t nb, double *ws_gsum, int64_t gsum_size,
+                                         float *mean, uint8_t *c2q, float *c1, cudaStream_t st);
 cudaError_t launch_dequantize(const uint8_t *codes, const uint8_t *c2q, const float *c1, const float *mean,
                               int64_t nb, const Nf4Levels &lv, uint16_t *out, cudaStream_t st);
+// merge.cu
+size_t merge_smem_bytes(int r);
+cudaError_t launch_merge_requantize(const qlora_nf4_weight &w, const uint16_t *A, const uint16_t *B, int r, float s,
+                                    const qlora_nf4_weight &out, uint16_t *w_merged, float *ws_absmax,
+                                    double *ws_gsum, int64_t gsum_size, const Nf4Levels &lv,
+                                    const Nf4Thresholds &thr, int *dev_err, unsigned long long timeout_ns,
+                                    cudaStream_t st);
 // adamw.cu
 using AdamwTensor = qlora_adamw_tensor;
 constexpr int kAdamwMaxTensors = QLORA_ADAMW_MAX_TENSORS;

@@ -66,6 +66,20 @@ __device__ __forceinline__ uint32_t bucket_code(float xh, const CodeBucket *tab)
   return static_cast<uint32_t>(e.base + (xh >= e.thr ? 1 : 0));
 }
 
+// Nearest level by counting thresholds (15 compares); for the rare blocks
+// whose absmax is too small for the reciprocal path.
+template <typename Thresholds>
+__device__ __forceinline__ uint32_t nf4_code(float xh, const Thresholds &t) {
+  uint32_t c = 0;
+#pragma unroll
+  for (int i = 0; i < 15; ++i) c += (xh >= t.t[i]) ? 1u : 0u;
+  return c;
+}
+
+// Blocks whose absmax is at least this use the reciprocal + corrected-quotient
+// path (exact there: see quotient_rn); smaller ones divide directly.
+constexpr float kFastQuotientMinAbsmax = 7.888609052210118e-31f;  // 2^-100
+
 // Same lookup in a table replicated once per lane ([bucket][lane]), so that 32
 // lanes looking up arbitrary buckets never share a bank.
 __device__ __forceinline__ uint32_t lane_bucket_code(float xh, const CodeBucket (*tab)[32], int lane) {

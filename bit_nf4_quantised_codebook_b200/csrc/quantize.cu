@@ -31,12 +31,6 @@ __device__ __forceinline__ uint32_t e4m3_from_f32_satfinite(float x) {
   return two & 0xFFu;
 }
 
-__device__ __forceinline__ uint32_t nf4_code(float xh, const Nf4Thresholds &t) {
-  uint32_t c = 0;
-#pragma unroll
-  for (int i = 0; i < 15; ++i) c += (xh >= t.t[i]) ? 1u : 0u;
-  return c;
-}
 
 // Streaming 16-byte load that does not keep the line in L1.
 __device__ __forceinline__ uint4 ld_stream_v4(const void *p) {
@@ -47,9 +41,28 @@ __device__ __forceinline__ uint4 ld_stream_v4(const void *p) {
   return v;
 }
 
-// Blocks whose absmax is at least this use the reciprocal + corrected-quotient
-// path (exact there: see nf4_quant.cuh); smaller ones divide directly.
-constexpr float kFastQuotientMinAbsmax = 7.888609052210118e-31f;  // 2^-100
+// Sum of s[0..255] by the pairwise tree (h = 128, 64, ..., 1: s[i] += s[i+h]);
+// called by all 256 threads, the sum is returned in thread 0.  Both the
+// quantiser and the group-sum pass of the adapter merge use it, so the block
+// constants of a group are always added in this one order.
+__device__ __forceinline__ double tree_sum256(double *s) {
+  __syncthreads();
+  const int t = threadIdx.x;
+  for (int h = 128; h >= 32; h >>= 1) {
+    if (t < h) s[t] = __dadd_rn(s[t], s[t + h]);
+    __syncthreads();
+  }
+  double v = 0.0;
+  if (t < 32) {
+    v = s[t];
+#pragma unroll
+    for (int h = 16; h >= 1; h >>= 1) {
+      const double o = __shfl_down_sync(0xFFFFFFFFu, v, h);
+      if (t < h) v = __dadd_rn(v, o);
+    }
+  }
+  return v;
+}
 
 // One CTA walks groups g = blockIdx.x, blockIdx.x + gridDim.x, ...; while it
 // codes one group the 16-byte loads of its next group are already in flight.
@@ -130,26 +143,26 @@ __global__ void __launch_bounds__(256, 2) k_quant_blocks(const uint16_t *__restr
       if (part == 0) s_sum[lb] = valid ? static_cast<double>(amax) : 0.0;
     }
     // group sum: pairwise tree over the 256 (zero-padded) block constants
-    __syncthreads();
-    const int t = threadIdx.x;
-    for (int h = 128; h >= 32; h >>= 1) {
-      if (t < h) s_sum[t] = __dadd_rn(s_sum[t], s_sum[t + h]);
-      __syncthreads();
-    }
-    if (t < 32) {
-      double v = s_sum[t];
-#pragma unroll
-      for (int h = 16; h >= 1; h >>= 1) {
-        const double o = __shfl_down_sync(0xFFFFFFFFu, v, h);
-        if (t < h) v = __dadd_rn(v, o);
-      }
-      if (t == 0) gsum[g] = v;
-    }
+    const double gs = tree_sum256(s_sum);
+    if (threadIdx.x == 0) gsum[g] = gs;
     __syncthreads();  // s_sum is reused by the next group
 #pragma unroll
     for (int pass = 0; pass < 8; ++pass) cur[pass] = nxt[pass];
   }
   if (bad && dev_err) atomicOr(dev_err, QLORA_DEVERR_NONFINITE);
+}
+
+// Group sums of float32 block constants that are already in memory (the
+// adapter merge writes them): one CTA per group, the same tree as above.
+__global__ void __launch_bounds__(256) k_group_sums(const float *__restrict__ absmax, int64_t nb,
+                                                     double *__restrict__ gsum) {
+  __shared__ double s_sum[256];
+  pdl_wait();
+  pdl_launch_dependents();
+  const int64_t b = static_cast<int64_t>(blockIdx.x) * 256 + threadIdx.x;
+  s_sum[threadIdx.x] = b < nb ? static_cast<double>(absmax[b]) : 0.0;
+  const double gs = tree_sum256(s_sum);
+  if (threadIdx.x == 0) gsum[blockIdx.x] = gs;
 }
 
 // Pairwise tree over the power-of-two padded group sums: for h = size/2, ..., 1
@@ -245,10 +258,21 @@ cudaError_t launch_quantize(const uint16_t *W, int64_t nb, uint8_t *codes, uint8
   cudaError_t e = launch_k(k_quant_blocks, dim3(static_cast<unsigned>(grid)), dim3(256), 0, st, 1, W, nb, codes,
                            ws_absmax, ws_gsum, thr, dev_err);
   if (e != cudaSuccess) return e;
-  e = launch_k(k_mean_tree, dim3(1), dim3(1024), 0, st, 1, ws_gsum, ng, gsum_size, nb, mean);
+  return launch_mean_and_double_quant(ws_absmax, nb, ws_gsum, gsum_size, mean, c2q, c1, st);
+}
+
+cudaError_t launch_mean_and_double_quant(const float *ws_absmax, int64_t nb, double *ws_gsum, int64_t gsum_size,
+                                         float *mean, uint8_t *c2q, float *c1, cudaStream_t st) {
+  const int64_t ng = (nb + 255) / 256;
+  cudaError_t e = launch_k(k_mean_tree, dim3(1), dim3(1024), 0, st, 1, ws_gsum, ng, gsum_size, nb, mean);
   if (e != cudaSuccess) return e;
-  return launch_k(k_double_quant, dim3(static_cast<unsigned>(ng)), dim3(256), 0, st, 1,
-                  static_cast<const float *>(ws_absmax), nb, static_cast<const float *>(mean), c2q, c1);
+  return launch_k(k_double_quant, dim3(static_cast<unsigned>(ng)), dim3(256), 0, st, 1, ws_absmax, nb,
+                  static_cast<const float *>(mean), c2q, c1);
+}
+
+cudaError_t launch_group_sums(const float *ws_absmax, int64_t nb, double *ws_gsum, cudaStream_t st) {
+  const int64_t ng = (nb + 255) / 256;
+  return launch_k(k_group_sums, dim3(static_cast<unsigned>(ng)), dim3(256), 0, st, 1, ws_absmax, nb, ws_gsum);
 }
 
 cudaError_t launch_dequantize(const uint8_t *codes, const uint8_t *c2q, const float *c1, const float *mean,

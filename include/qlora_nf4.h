@@ -80,7 +80,7 @@ typedef struct qlora_nf4_weight {
   float *mean;       /* 1 float       */
 } qlora_nf4_weight;
 
-enum { QLORA_OP_QUANTIZE = 0, QLORA_OP_FORWARD = 1, QLORA_OP_BACKWARD = 2 };
+enum { QLORA_OP_QUANTIZE = 0, QLORA_OP_FORWARD = 1, QLORA_OP_BACKWARD = 2, QLORA_OP_MERGE = 3 };
 
 /* Human-readable name of a status code (static string). */
 const char *qlora_status_string(qlora_status st);
@@ -107,7 +107,7 @@ qlora_status qlora_nf4_sizes(int64_t N, int64_t K, size_t *codes_bytes, size_t *
 
 /*
  * Workspace bytes an operation needs (op = QLORA_OP_*; M and r are ignored for
- * QLORA_OP_QUANTIZE).  The caller allocates it (16-byte aligned) and passes it
+ * QLORA_OP_QUANTIZE and QLORA_OP_MERGE).  The caller allocates it (16-byte aligned) and passes it
  * to the call; it holds no state between calls.
  */
 qlora_status qlora_workspace_size(int op, int64_t M, int64_t N, int64_t K, int r, size_t *bytes);
@@ -118,8 +118,9 @@ qlora_status qlora_workspace_size(int op, int64_t M, int64_t N, int64_t K, int r
  * Per block: c2 = max|w| (float32); x = float32(w / c2); code = nearest level
  * (ties to the lower index; an all-zero block gives the zero level, 7).
  * Second level: mu = mean of all c2 in a fixed order (per group of 256 blocks
- * a sequential float64 sum, then a power-of-two pairwise tree; float64 divide
- * by the block count, rounded to float32); dev = float32(c2 - mu);
+ * a float64 pairwise tree — h = 128, 64, ..., 1: a[i] += a[i+h] — then the same
+ * tree over the group sums zero-padded to a power of two; float64 divide by
+ * the block count, rounded to float32); dev = float32(c2 - mu);
  * S_g = float32(max|dev| over the group / 448); e = E4M3(dev / S_g) with
  * round-to-nearest-even and saturation (S_g = 0 gives e = 0).
  * Writes out->codes, out->c2q, out->c1, out->mean.  A non-finite weight sets
@@ -156,6 +157,36 @@ qlora_status qlora_quantize_noalloc(const uint16_t *W, const qlora_nf4_weight *o
  * W_out: device, N*K bfloat16.
  */
 qlora_status qlora_dequantize(const qlora_nf4_weight *w, uint16_t *W_out, void *stream);
+
+/*
+ * qlora_merge_requantize — merge a trained adapter into the quantised base and
+ * requantise ("QLoRA: quantising the part you are not training", addaly.com,
+ * §What it costs: merging into the quantised base means requantising).  The
+ * layer computes X·Ŵᵀ + s·(X·A)·B (§The QLoRA layer, end to end,
+ * intuitivepapers.ai), so the merged weight is
+ *   W_eff[n][k] = bf16_rn( float32( ŵ[n][k] + s · sum_j A[k][j]·B[j][n] ) )
+ * with ŵ = doubleDequant(w), the sum accumulated in float32 on the tensor
+ * cores (order unspecified), and one float32 rounding of ŵ + s·sum (a fused
+ * multiply-add).  W_eff is then quantised exactly as qlora_quantize does.
+ * w   : the stored weight (device buffers), N x K.
+ * A   : device, K x r bfloat16 row-major; B: device, r x N bfloat16 row-major
+ *       (the layer's adapter); r % 8 == 0, r <= 256; N % 8 == 0.
+ * s   : the adapter scale alpha / r.
+ * out : the new stored weight, same N, K.  It may be w itself (in place);
+ *       otherwise none of its buffers may overlap any of w's.
+ * W_merged : device N x K bfloat16 (nullable): receives W_eff; must not
+ *       overlap w or out.
+ * ws  : qlora_workspace_size(QLORA_OP_MERGE, 0, N, K, r) bytes (the
+ *       quantiser's workspace).
+ * A non-finite merged weight sets QLORA_DEVERR_NONFINITE in *dev_err; a
+ * pipeline wait that runs out sets QLORA_DEVERR_TIMEOUT (outputs then
+ * unspecified).  Errors: QLORA_ERR_INVALID_ARG (null pointer, shape mismatch,
+ * partial overlap of out and w), QLORA_ERR_UNSUPPORTED_SHAPE, QLORA_ERR_MISALIGNED,
+ * QLORA_ERR_WORKSPACE, QLORA_ERR_NO_DEVICE, QLORA_ERR_CUDA.
+ */
+qlora_status qlora_merge_requantize(const qlora_nf4_weight *w, const uint16_t *A, const uint16_t *B, int r,
+                                    float s, const qlora_nf4_weight *out, uint16_t *W_merged, void *ws,
+                                    size_t ws_bytes, int *dev_err, void *stream);
 
 /*
  * qlora_linear_forward — §LoRA and §The QLoRA layer, end to end (forward).
@@ -239,7 +270,8 @@ uint64_t qlora_kernel_launch_count(void);
  * immediately before / after launching the dequant GEMM that produces Y (the
  * small-M kernel when M <= 64), and every
  * qlora_linear_backward records bwd_begin / bwd_end around the fused dequant
- * GEMM that produces dX.  Passing all NULL disables the hooks.  The setting is
+ * GEMM that produces dX; every qlora_merge_requantize records fwd_begin /
+ * fwd_end around its merge-and-code kernel.  Passing all NULL disables the hooks.  The setting is
  * process-wide and not thread-safe.
  */
 qlora_status qlora_set_timing_events(void *fwd_begin, void *fwd_end, void *bwd_begin, void *bwd_end);

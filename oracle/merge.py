@@ -43,11 +43,17 @@ _U = 2.0 ** -53          # unit roundoff of float64
 
 
 def _exact_f32(w: float, s: float, a_row: np.ndarray, b_col: np.ndarray) -> np.float32:
-    """float32 of w + s·sum(a_row·b_col), computed with rationals."""
-    acc = Fraction(0)
-    for x, y in zip(a_row.tolist(), b_col.tolist()):
-        acc += Fraction(x) * Fraction(y)
-    return _round_fraction_to_f32(Fraction(w) + Fraction(s) * acc)
+    """float32 of w + s·sum(a_row·b_col), from the exact value.
+
+    Each term s·a·b is exact in float64: s has 24 significant bits, a and b 8
+    each (bfloat16), so the product needs at most 40, and its exponent stays
+    far inside float64's range.  The terms are then added exactly as integers
+    over their common power-of-two denominator."""
+    ratios = [w.as_integer_ratio()] + [(s * x * y).as_integer_ratio()
+                                       for x, y in zip(a_row.tolist(), b_col.tolist())]
+    den = max(d for _, d in ratios)                 # every denominator is a power of two
+    num = sum(n * (den // d) for n, d in ratios)
+    return _round_fraction_to_f32(Fraction(num, den))
 
 
 def merged_weight(w_hat_bits: np.ndarray, a_bits: np.ndarray, b_bits: np.ndarray, s: float) -> np.ndarray:

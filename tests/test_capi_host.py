@@ -81,6 +81,35 @@ def test_validation_errors(api):
     assert api.lib().qlora_status_string(3) == b"pointer not 16-byte aligned"
 
 
+def test_merge_validation(api):
+    """qlora_merge_requantize rejects bad arguments before any launch (1 = invalid
+    argument, 2 = unsupported shape, 3 = misaligned); every case here fails
+    before the device is touched."""
+    L = api.lib()
+    W = api._Weight
+    w = W(16, 128, 4096, 8192, 12288, 16384)             # codes 1 KiB, c2q 32 B, c1 4 B, mean
+    out = W(16, 128, 65536, 69632, 73728, 77824)
+    f = ctypes.c_float(0.25)
+    ok = dict(A=1 << 20, B=1 << 21, r=16)
+
+    def call(w_=w, out_=out, A=ok["A"], B=ok["B"], r=ok["r"], wm=None):
+        return L.qlora_merge_requantize(ctypes.byref(w_), A, B, r, f, ctypes.byref(out_), wm, 1 << 22, 1 << 20,
+                                        None, None)
+
+    assert call(out_=W(24, 128, 65536, 69632, 73728, 77824)) == 1   # shape mismatch
+    assert call(A=None) == 1
+    assert call(B=None) == 1
+    assert call(r=0) == 1
+    assert call(r=12) == 2
+    assert call(r=264) == 2
+    assert call(w_=W(12, 128, 4096, 8192, 12288, 16384), out_=W(12, 128, 65536, 69632, 73728, 77824)) == 2
+    assert call(A=(1 << 20) + 8) == 3
+    assert call(wm=4104) == 3
+    assert call(out_=W(16, 128, 4096 + 512, 69632, 73728, 77824)) == 1   # partial overlap of codes
+    assert call(out_=W(16, 128, 65536, 4096, 73728, 77824)) == 1         # out.c2q inside w.codes
+    assert call(wm=8192 - 16) == 1                                        # W_merged over w's buffers
+
+
 def test_product_path_has_no_cpu_fallback():
     """The binding never imports the oracle; the package refuses to run without the library."""
     pkg = os.path.join(ROOT, "bit_nf4_quantised_codebook_b200")
