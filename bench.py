@@ -645,6 +645,10 @@ def run_merge(args):
     torch.cuda.synchronize()
     nj = len(MERGE_SHAPES)
     ev = [[[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(nj)] for _ in range(args.steps)]
+    for row in ev:  # torch creates the CUDA event at its first record; the library records them afterwards
+        for pair in row:
+            for e in pair:
+                e.record()
     gpu_id = None
     try:
         gpu_id = "GPU-" + str(torch.cuda.get_device_properties(local).uuid)
