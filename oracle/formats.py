@@ -23,8 +23,8 @@ Readings (also listed in the design doc):
     sign + 3-bit layouts, E2M1 (exponent bias 1, one subnormal step: 0, 0.5,
     1, 1.5, 2, 3, 4, 6) and E3M0 (bias 3, no mantissa: 0, 0.25, ..., 16),
     each divided by its largest value so the block's absmax maps to +-1; their
-    two zeros (+0, -0) both become 0 and the nearest-level rule with ties to
-    the lower index picks the first;
+    two zeros (+0, -0) both become the level +0, and the nearest-level rule
+    with ties to the lower index only ever picks the first of the two;
   * every code book is used like NF4: x_hat = float32(w / absmax), nearest
     level of the float32 table, ties to the lower index;
   * block sizes 32, 64, 128 and 256 run along the flattened tensor like the
@@ -85,7 +85,8 @@ def codebook(name: str) -> np.ndarray:
     else:
         raise ValueError(name)
     pos = pos / pos.max()
-    v = np.sort(np.concatenate([-pos, pos]))          # holds 0 twice (from +0 and -0)
+    nz = pos[pos > 0]
+    v = np.concatenate([-nz[::-1], [0.0, 0.0], nz])  # the layout's +0 and -0, both stored as +0
     return v.astype(_F32)
 
 

@@ -34,6 +34,7 @@ def test_float4_code_books_are_the_layouts_values():
         want = np.sort(np.concatenate([-pos, pos])).astype(np.float32)
         assert np.array_equal(lv, want), name
         assert lv[0] == -1 and lv[-1] == 1 and np.count_nonzero(lv == 0) == 2
+        assert not np.signbit(lv[lv == 0]).any()
 
 
 def test_int4_grid():
@@ -65,6 +66,10 @@ def test_nearest_level_by_midpoints(cb):
     xh = nf4.bf16_to_f64(to_bf16_bits(w))
     want = np.array([lv[np.count_nonzero(v > m)] for v in xh])
     assert np.array_equal(lv[codes], want.astype(np.float32))
+    # of two equal levels only the first is ever used (ties go to the lower index)
+    for i in range(15):
+        if lv[i] == lv[i + 1]:
+            assert not np.any(codes == i + 1)
 
 
 def test_main_format_is_the_special_case():
