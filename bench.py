@@ -767,6 +767,174 @@ def cpu_baseline_merge(min_seconds: float = 10.0) -> dict:
                                         f"q projection (float64 numpy); {tot_t:.1f} s"}
 
 
+FORMAT_CODEBOOKS = ("nf4", "int4", "fp4_e2m1", "fp4_e3m0")
+FORMAT_BLOCKS = (32, 64, 128, 256)
+FORMAT_DQ = ("none", "e4m3", "int8")
+
+
+def format_stored_bytes(n: int, k: int, block: int, dq: str) -> int:
+    nb = n * k // block
+    return n * k // 2 + (4 * nb if dq == "none" else nb + 4 * (-(-nb // 256)) + 4)
+
+
+def format_step_bytes(n: int, k: int, block: int, dq: str) -> int:
+    """Algorithmic bytes of one study point: quantise (read W, write the stored
+    form), dequantise (read it, write W_hat), error (read W and W_hat)."""
+    st = format_stored_bytes(n, k, block, dq)
+    return (2 * n * k + st) + (st + 2 * n * k) + 4 * n * k
+
+
+def run_formats(args):
+    """The format study: the 4096 x 4096 weight (N(0, 0.02) with 0.1% t(3)
+    outliers) quantised, dequantised and measured in every code book x block
+    size x constant treatment; a step is the 48 round trips."""
+    import itertools
+    import torch
+    import torch.distributed as dist
+    from datetime import timedelta
+    from bit_nf4_quantised_codebook_b200 import api, inputs
+
+    world, rank, local = _dist()
+    torch.cuda.set_device(local)
+    if world > 1:
+        dist.init_process_group("nccl", timeout=timedelta(seconds=120), device_id=torch.device("cuda", local))
+    api.lib()
+    dev = torch.device("cuda", local)
+    N = K = 4096
+    wbits = inputs.weight_bf16(N, K, 0.02, 0, 0.001)
+    ncopy = 4  # 4 x 33.5 MB of W in rotation (> L2)
+    Ws = [api.bits_to_tensor(wbits, dev) for _ in range(ncopy)]
+    fmts = list(itertools.product(FORMAT_CODEBOOKS, FORMAT_BLOCKS, FORMAT_DQ))
+    outs = [api.alloc_format_weight(N, K, cb, b, dq, dev) for cb, b, dq in fmts]
+    what = torch.empty(N, K, dtype=torch.bfloat16, device=dev)
+    stats = torch.empty(len(fmts), 3, dtype=torch.float64, device=dev)
+    ws = torch.empty(1 << 24, dtype=torch.uint8, device=dev)
+    err = api.new_error_word(dev)
+    step_bytes = sum(format_step_bytes(N, K, b, dq) for _, b, dq in fmts)
+
+    def step(i, W=None):
+        W = Ws[i % ncopy] if W is None else W
+        for j, (cb, b, dq) in enumerate(fmts):
+            api.qlora_quantize_format(W, cb, b, dq, out=outs[j], ws=ws, dev_err=err)
+            api.qlora_dequantize_format(outs[j], what)
+            api.qlora_quant_error(W, what, stats[j])
+
+    for i in range(args.warmup):
+        step(i)
+    torch.cuda.synchronize()
+    gpu_id = None
+    try:
+        gpu_id = "GPU-" + str(torch.cuda.get_device_properties(local).uuid)
+    except Exception:
+        pass
+    sampler = ClockSampler(gpu_id)
+    sampler.start()
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    launches0 = api.qlora_kernel_launch_count()
+    sampler.mark_start()
+    t0 = torch.cuda.Event(enable_timing=True)
+    t1 = torch.cuda.Event(enable_timing=True)
+    t0.record()
+    for i in range(args.steps):
+        step(i)
+    t1.record()
+    torch.cuda.synchronize()
+    sampler.mark_end()
+    launches = api.qlora_kernel_launch_count() - launches0
+    # the NF4 / 64 / E4M3 quantisation alone (block kernel + second quantisation)
+    j0 = fmts.index(("nf4", 64, "e4m3"))
+    q_ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    for i in range(args.steps):
+        q_ev[i][0].record()
+        api.qlora_quantize_format(Ws[i % ncopy], "nf4", 64, "e4m3", out=outs[j0], ws=ws, dev_err=err)
+        q_ev[i][1].record()
+    torch.cuda.synchronize()
+    clocks = sampler.stop()
+    ms = t0.elapsed_time(t1)
+    q_ms = sum(a.elapsed_time(b) for a, b in q_ev) / args.steps
+    if world > 1:
+        ms = max_over_ranks(ms, dev)
+    if int(err[0].item()) != 0:
+        raise RuntimeError(f"device error word {int(err[0].item())}")
+    ms_step = ms / args.steps
+    value = whole_job_rate(step_bytes, world, ms_step * 1e-3) / 1e9
+    st = stats.cpu().numpy()
+    curves = []
+    for j, (cb, b, dq) in enumerate(fmts):
+        curves.append({"codebook": cb, "block": b, "dq": dq,
+                       "bits_per_weight": round(8 * format_stored_bytes(N, K, b, dq) / (N * K), 4),
+                       "rel_fro": round(float((st[j, 0] / st[j, 1]) ** 0.5), 5), "max_abs": float(st[j, 2])})
+
+    # end to end: W host -> device, the 48 round trips, the statistics device -> host
+    e2e_steps = max(3, min(20, args.steps // 10))
+    hw = Ws[0].cpu().pin_memory()
+    hs = torch.empty_like(stats, device="cpu").pin_memory()
+    dw = torch.empty_like(Ws[0])
+    torch.cuda.synchronize()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for i in range(e2e_steps):
+        dw.copy_(hw, non_blocking=True)
+        step(i, dw)
+        hs.copy_(stats, non_blocking=True)
+    e1.record()
+    torch.cuda.synchronize()
+    e2e_ms = e0.elapsed_time(e1) / e2e_steps
+
+    hbm, _, _, peak_src = _peaks()
+    q_bytes = 2 * N * K + format_stored_bytes(N, K, 64, "e4m3")
+    achieved = q_bytes / (q_ms * 1e-3) / 1e9
+    line = {
+        "metric": "format study throughput (quantise + dequantise + error, all formats)",
+        "value": round(value, 2), "unit": "GB/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_step, 5),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32",
+        "data": "synthetic (seeded numpy N(0,0.02) with 0.1% 0.2*t(3) outliers, rounded to bf16)",
+        "config": {"workload": "NF4 / Int4 / FP4 E2M1 / FP4 E3M0 x blocks 32-256 x constants float32/E4M3/int8 "
+                               "on a 4096x4096 weight", "formats": len(fmts),
+                   "parallelism": f"replicas x{world} (no shard)",
+                   "l2": f"{ncopy} copies of W in rotation ({ncopy * 2 * N * K / 1e6:.0f} MB > L2)"},
+        "curves": curves,
+        "kernels": {"quantize_nf4_64_e4m3_ms": round(q_ms, 5)},
+        "roofline": {"kernel": "k_quant_format<64> + second quantisation (NF4, E4M3)", "bound": "hbm",
+                     "achieved": round(achieved, 1), "peak": hbm, "unit": "GB/s", "frac": round(achieved / hbm, 4),
+                     "peak_source": f"{peak_src} HBM copy", "traffic": None,
+                     "traffic_unit": "bytes per launch (ncu dram read+write)"},
+        "e2e": {"value": round(step_bytes / (e2e_ms * 1e-3) / 1e9, 2), "unit": "GB/s",
+                "h2d_bytes_per_step": 2 * N * K, "d2h_bytes_per_step": stats.numel() * 8, "steps": e2e_steps},
+        "gpu_launches": int(launches),
+        "clocks": clocks,
+    }
+    if world == 1 and rank == 0 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline_formats(wbits[:256])
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+def cpu_baseline_formats(wbits, min_seconds: float = 10.0) -> dict:
+    """The oracle's round trip in every format on a slice of the weight."""
+    import itertools
+    from oracle import formats as F
+    n, k = wbits.shape
+    fmts = list(itertools.product(FORMAT_CODEBOOKS, FORMAT_BLOCKS, FORMAT_DQ))
+    tot_t, reps = 0.0, 0
+    while tot_t < min_seconds or reps == 0:
+        t = time.perf_counter()
+        for cb, b, dq in fmts:
+            F.error_stats(wbits, F.dequantize_q(F.quantize(wbits, cb, b, dq)))
+        tot_t += time.perf_counter() - t
+        reps += 1
+    by = reps * sum(format_step_bytes(n, k, b, dq) for _, b, dq in fmts)
+    return {"value": round(by / tot_t / 1e9, 6), "unit": "GB/s", "cores": os.cpu_count(), "kind": "oracle",
+            "sample": f"{reps} x the 48 round trips on {n} of the 4096 rows (float64 numpy); {tot_t:.1f} s"}
+
+
 def cpu_baseline_adamw(min_seconds: float = 10.0) -> dict:
     """The oracle's AdamW step on 2^20 parameters, repeated; bytes as on the GPU."""
     import numpy as np
@@ -882,7 +1050,7 @@ def main():
     ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--workload", choices=["proj7b", "smallm", "adamw", "merge"], default="proj7b")
+    ap.add_argument("--workload", choices=["proj7b", "smallm", "adamw", "merge", "formats"], default="proj7b")
     ap.add_argument("--n", type=int, default=8192, help="smallm: W rows (8192 or 28672)")
     ap.add_argument("--m", type=int, default=16, help="smallm: tokens (1..64)")
     args = ap.parse_args()
@@ -894,6 +1062,8 @@ def main():
         run_adamw(args)
     elif args.workload == "merge":
         run_merge(args)
+    elif args.workload == "formats":
+        run_formats(args)
     else:
         run_ours(args)
 

@@ -18,12 +18,16 @@ LIB_PATH = os.path.join(_PKG, "libqlora_nf4.so")
 
 QLORA_OP_QUANTIZE, QLORA_OP_FORWARD, QLORA_OP_BACKWARD, QLORA_OP_MERGE = 0, 1, 2, 3
 QLORA_DEVERR_NONFINITE, QLORA_DEVERR_TIMEOUT = 1, 2
+CODEBOOKS = {"nf4": 0, "int4": 1, "fp4_e2m1": 2, "fp4_e3m0": 3}
+DQ_MODES = {"none": 0, "e4m3": 1, "int8": 2}
 
 EXPORTED = [
     "qlora_status_string", "qlora_build_codebook", "qlora_nf4_sizes", "qlora_workspace_size",
     "qlora_quantize", "qlora_dequantize", "qlora_linear_forward", "qlora_linear_backward",
     "qlora_kernel_launch_count", "qlora_set_timing_events", "qlora_quantize_noalloc",
     "qlora_selftest_bounded_wait", "qlora_adamw_step", "qlora_merge_requantize",
+    "qlora_format_codebook", "qlora_format_sizes", "qlora_format_workspace_size", "qlora_quantize_format",
+    "qlora_dequantize_format", "qlora_quant_error",
 ]
 
 
@@ -39,6 +43,15 @@ class _Weight(ctypes.Structure):
 class _AdamwTensor(ctypes.Structure):
     _fields_ = [("param", ctypes.c_void_p), ("param_bf16", ctypes.c_void_p), ("grad", ctypes.c_void_p),
                 ("m", ctypes.c_void_p), ("v", ctypes.c_void_p), ("n", ctypes.c_int64)]
+
+
+class _Format(ctypes.Structure):
+    _fields_ = [("codebook", ctypes.c_int), ("block", ctypes.c_int), ("dq", ctypes.c_int)]
+
+
+class _QWeight(ctypes.Structure):
+    _fields_ = [("N", ctypes.c_int64), ("K", ctypes.c_int64), ("fmt", _Format), ("codes", ctypes.c_void_p),
+                ("consts", ctypes.c_void_p), ("c1", ctypes.c_void_p), ("mean", ctypes.c_void_p)]
 
 
 _lib = None
@@ -69,6 +82,12 @@ def lib() -> ctypes.CDLL:
         L.qlora_quantize_noalloc.argtypes = [vp, ctypes.POINTER(_Weight), vp, vp]
         L.qlora_selftest_bounded_wait.argtypes = [ctypes.c_uint, vp, vp, vp]
         L.qlora_adamw_step.argtypes = [ctypes.POINTER(_AdamwTensor), i32, f32, f32, f32, f32, f32, i64, vp]
+        L.qlora_format_codebook.argtypes = [i32, vp, vp]
+        L.qlora_format_sizes.argtypes = [ctypes.POINTER(_Format), i64, i64, vp, vp, vp]
+        L.qlora_format_workspace_size.argtypes = [ctypes.POINTER(_Format), i64, i64, vp]
+        L.qlora_quantize_format.argtypes = [vp, ctypes.POINTER(_QWeight), vp, sz, vp, vp]
+        L.qlora_dequantize_format.argtypes = [ctypes.POINTER(_QWeight), vp, vp]
+        L.qlora_quant_error.argtypes = [vp, vp, i64, vp, vp]
         L.qlora_merge_requantize.argtypes = [ctypes.POINTER(_Weight), vp, vp, i32, f32, ctypes.POINTER(_Weight),
                                              vp, vp, sz, vp, vp]
         for name in EXPORTED[1:]:
@@ -189,6 +208,87 @@ def qlora_dequantize(w: NF4Weight, out: torch.Tensor | None = None) -> torch.Ten
     s = w.c_struct()
     _check(lib().qlora_dequantize(ctypes.byref(s), out.data_ptr(), _stream()), "qlora_dequantize")
     return out
+
+
+@dataclass
+class FormatWeight:
+    """A weight stored in one of the format variants (code book, block size,
+    treatment of the block constants)."""
+    N: int
+    K: int
+    codebook: str
+    block: int
+    dq: str
+    codes: torch.Tensor            # uint8 [N*K/2]
+    consts: torch.Tensor           # float32 [N*K/block] (dq "none") or uint8 [N*K/block]
+    c1: torch.Tensor | None        # float32 [ceil(N*K/block/256)]
+    mean: torch.Tensor | None      # float32 [4] (element 0)
+
+    def c_fmt(self) -> _Format:
+        return _Format(CODEBOOKS[self.codebook], self.block, DQ_MODES[self.dq])
+
+    def c_struct(self) -> _QWeight:
+        return _QWeight(self.N, self.K, self.c_fmt(), self.codes.data_ptr(), self.consts.data_ptr(), _ptr(self.c1),
+                        _ptr(self.mean))
+
+    def nbytes(self) -> int:
+        return (self.codes.numel() + self.consts.numel() * self.consts.element_size()
+                + (0 if self.c1 is None else 4 * self.c1.numel() + 4))
+
+
+def qlora_format_codebook(codebook: str) -> tuple[list[float], list[float]]:
+    lv = (ctypes.c_float * 16)()
+    th = (ctypes.c_float * 15)()
+    _check(lib().qlora_format_codebook(CODEBOOKS[codebook], lv, th), "qlora_format_codebook")
+    return list(lv), list(th)
+
+
+def alloc_format_weight(N: int, K: int, codebook: str, block: int, dq: str, device=None) -> FormatWeight:
+    f = _Format(CODEBOOKS[codebook], block, DQ_MODES[dq])
+    a, b, c = ctypes.c_size_t(), ctypes.c_size_t(), ctypes.c_size_t()
+    _check(lib().qlora_format_sizes(ctypes.byref(f), N, K, ctypes.byref(a), ctypes.byref(b), ctypes.byref(c)),
+           "qlora_format_sizes")
+    dev = device or torch.device("cuda")
+    consts = (torch.empty(b.value // 4, dtype=torch.float32, device=dev) if dq == "none"
+              else torch.empty(b.value, dtype=torch.uint8, device=dev))
+    c1 = None if dq == "none" else torch.empty(max(1, c.value // 4), dtype=torch.float32, device=dev)
+    mean = None if dq == "none" else torch.zeros(4, dtype=torch.float32, device=dev)
+    return FormatWeight(N, K, codebook, block, dq, torch.empty(a.value, dtype=torch.uint8, device=dev), consts, c1,
+                        mean)
+
+
+def qlora_quantize_format(W: torch.Tensor, codebook: str, block: int, dq: str, out: FormatWeight | None = None,
+                          ws: torch.Tensor | None = None, dev_err: torch.Tensor | None = None) -> FormatWeight:
+    N, K = W.shape
+    _need(W, torch.bfloat16, (N, K), "W")
+    out = out or alloc_format_weight(N, K, codebook, block, dq, W.device)
+    f = out.c_fmt()
+    need = ctypes.c_size_t()
+    _check(lib().qlora_format_workspace_size(ctypes.byref(f), N, K, ctypes.byref(need)),
+           "qlora_format_workspace_size")
+    if ws is None:
+        ws = torch.empty(max(16, need.value), dtype=torch.uint8, device=W.device)
+    s = out.c_struct()
+    _check(lib().qlora_quantize_format(W.data_ptr(), ctypes.byref(s), ws.data_ptr(), ws.numel(), _ptr(dev_err),
+                                       _stream()), "qlora_quantize_format")
+    return out
+
+
+def qlora_dequantize_format(w: FormatWeight, out: torch.Tensor | None = None) -> torch.Tensor:
+    out = out if out is not None else torch.empty((w.N, w.K), dtype=torch.bfloat16, device=w.codes.device)
+    _need(out, torch.bfloat16, (w.N, w.K), "W_out")
+    s = w.c_struct()
+    _check(lib().qlora_dequantize_format(ctypes.byref(s), out.data_ptr(), _stream()), "qlora_dequantize_format")
+    return out
+
+
+def qlora_quant_error(W: torch.Tensor, W_hat: torch.Tensor, stats: torch.Tensor | None = None) -> torch.Tensor:
+    """Device float64 [3]: sum (w - w_hat)^2, sum w^2, max |w - w_hat|."""
+    _need(W_hat, torch.bfloat16, tuple(W.shape), "W_hat")
+    stats = stats if stats is not None else torch.empty(3, dtype=torch.float64, device=W.device)
+    _check(lib().qlora_quant_error(W.data_ptr(), W_hat.data_ptr(), W.numel(), stats.data_ptr(), _stream()),
+           "qlora_quant_error")
+    return stats
 
 
 def qlora_merge_requantize(w: NF4Weight, A: torch.Tensor, B: torch.Tensor, s: float, out: NF4Weight | None = None,

@@ -20,7 +20,7 @@ ROOT = os.path.dirname(PKG)
 CSRC = os.path.join(PKG, "csrc")
 BUILD = os.path.join(ROOT, "_build")
 LIB = os.path.join(PKG, "libqlora_nf4.so")
-SOURCES = ["codebook.cpp", "quantize.cu", "quantize_noalloc.cu", "linear.cu", "merge.cu", "adamw.cu", "selftest.cu",
+SOURCES = ["codebook.cpp", "quantize.cu", "quantize_noalloc.cu", "linear.cu", "merge.cu", "formats.cu", "adamw.cu", "selftest.cu",
            "capi.cu"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 

@@ -346,6 +346,113 @@ qlora_status qlora_merge_requantize(const qlora_nf4_weight *w, const uint16_t *A
   return e == cudaSuccess ? QLORA_OK : QLORA_ERR_CUDA;
 }
 
+// ---------------------------------------------------------------- format variants
+static qlora_status check_format(const qlora_format *f) {
+  if (!f || f->codebook < QLORA_CB_NF4 || f->codebook > QLORA_CB_FP4_E3M0 || f->dq < QLORA_DQ_NONE ||
+      f->dq > QLORA_DQ_INT8)
+    return QLORA_ERR_INVALID_ARG;
+  if (f->block != 32 && f->block != 64 && f->block != 128 && f->block != 256) return QLORA_ERR_UNSUPPORTED_SHAPE;
+  return QLORA_OK;
+}
+
+static qlora_status check_format_shape(const qlora_format *f, int64_t N, int64_t K) {
+  qlora_status st = check_format(f);
+  if (st != QLORA_OK) return st;
+  if (N < 1 || K < 1) return QLORA_ERR_INVALID_ARG;
+  if (K % f->block != 0 || N > (1ll << 30) || K > (1ll << 30) || N * K > (1ll << 40))
+    return QLORA_ERR_UNSUPPORTED_SHAPE;
+  return QLORA_OK;
+}
+
+static qlora_status check_qweight(const qlora_qweight *w) {
+  if (!w) return QLORA_ERR_INVALID_ARG;
+  qlora_status st = check_format_shape(&w->fmt, w->N, w->K);
+  if (st != QLORA_OK) return st;
+  if (!w->codes || !w->consts || (w->fmt.dq != QLORA_DQ_NONE && (!w->c1 || !w->mean))) return QLORA_ERR_INVALID_ARG;
+  if (!aligned16(w->codes) || !aligned16(w->consts) || (w->c1 && !aligned16(w->c1)) ||
+      (w->mean && !aligned16(w->mean)))
+    return QLORA_ERR_MISALIGNED;
+  return QLORA_OK;
+}
+
+// Workspace of the format quantiser: float32 absmax per block, then the
+// power-of-two padded float64 group sums.
+static void format_ws_layout(int64_t nb, size_t *off_gsum, int64_t *gsum_size, size_t *bytes) {
+  const int64_t ng = (nb + 255) / 256;
+  int64_t size = 1;
+  while (size < ng) size *= 2;
+  *off_gsum = align256(static_cast<size_t>(nb) * 4);
+  *gsum_size = size;
+  *bytes = align256(*off_gsum + static_cast<size_t>(size) * 8);
+}
+
+qlora_status qlora_format_codebook(int codebook, float levels[16], float thresholds[15]) {
+  return build_format_codebook_f32(codebook, levels, thresholds) ? QLORA_OK : QLORA_ERR_INVALID_ARG;
+}
+
+qlora_status qlora_format_sizes(const qlora_format *fmt, int64_t N, int64_t K, size_t *codes_bytes,
+                                size_t *consts_bytes, size_t *c1_bytes) {
+  qlora_status st = check_format_shape(fmt, N, K);
+  if (st != QLORA_OK) return st;
+  const int64_t nb = N * K / fmt->block;
+  if (codes_bytes) *codes_bytes = static_cast<size_t>(N * K / 2);
+  if (consts_bytes) *consts_bytes = static_cast<size_t>(nb) * (fmt->dq == QLORA_DQ_NONE ? 4 : 1);
+  if (c1_bytes) *c1_bytes = fmt->dq == QLORA_DQ_NONE ? 0 : static_cast<size_t>((nb + 255) / 256) * 4;
+  return QLORA_OK;
+}
+
+qlora_status qlora_format_workspace_size(const qlora_format *fmt, int64_t N, int64_t K, size_t *bytes) {
+  if (!bytes) return QLORA_ERR_INVALID_ARG;
+  qlora_status st = check_format_shape(fmt, N, K);
+  if (st != QLORA_OK) return st;
+  size_t off;
+  int64_t size;
+  format_ws_layout(N * K / fmt->block, &off, &size, bytes);
+  return QLORA_OK;
+}
+
+qlora_status qlora_quantize_format(const uint16_t *W, const qlora_qweight *w, void *ws, size_t ws_bytes,
+                                   int *dev_err, void *stream) {
+  if (!W) return QLORA_ERR_INVALID_ARG;
+  qlora_status st = check_qweight(w);
+  if (st != QLORA_OK) return st;
+  if (!aligned16(W)) return QLORA_ERR_MISALIGNED;
+  size_t off_gsum, need;
+  int64_t gsum_size;
+  format_ws_layout(w->N * w->K / w->fmt.block, &off_gsum, &gsum_size, &need);
+  if (!ws || ws_bytes < need) return QLORA_ERR_WORKSPACE;
+  if (!aligned16(ws)) return QLORA_ERR_MISALIGNED;
+  if (!device_ok()) return QLORA_ERR_NO_DEVICE;
+  float levels[16], thr[15];
+  build_format_codebook_f32(w->fmt.codebook, levels, thr);
+  uint8_t *w8 = static_cast<uint8_t *>(ws);
+  const cudaError_t e = launch_quantize_format(W, *w, levels, thr, reinterpret_cast<float *>(w8),
+                                               reinterpret_cast<double *>(w8 + off_gsum), gsum_size, dev_err,
+                                               static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? QLORA_OK : QLORA_ERR_CUDA;
+}
+
+qlora_status qlora_dequantize_format(const qlora_qweight *w, uint16_t *W_out, void *stream) {
+  qlora_status st = check_qweight(w);
+  if (st != QLORA_OK) return st;
+  if (!W_out) return QLORA_ERR_INVALID_ARG;
+  if (!aligned16(W_out)) return QLORA_ERR_MISALIGNED;
+  if (!device_ok()) return QLORA_ERR_NO_DEVICE;
+  float levels[16];
+  build_format_codebook_f32(w->fmt.codebook, levels, nullptr);
+  const cudaError_t e = launch_dequantize_format(*w, levels, W_out, static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? QLORA_OK : QLORA_ERR_CUDA;
+}
+
+qlora_status qlora_quant_error(const uint16_t *W, const uint16_t *W_hat, int64_t n, double *stats, void *stream) {
+  if (!W || !W_hat || !stats || n < 1) return QLORA_ERR_INVALID_ARG;
+  if (!aligned16(W) || !aligned16(W_hat) || (reinterpret_cast<uintptr_t>(stats) & 7u) != 0)
+    return QLORA_ERR_MISALIGNED;
+  if (!device_ok()) return QLORA_ERR_NO_DEVICE;
+  const cudaError_t e = launch_quant_error(W, W_hat, n, stats, device_sms(), static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? QLORA_OK : QLORA_ERR_CUDA;
+}
+
 static LaunchCtx make_ctx(int *dev_err, void *stream) {
   Globals &g = globals();
   LaunchCtx c;

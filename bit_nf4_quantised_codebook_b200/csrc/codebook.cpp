@@ -108,21 +108,54 @@ void build_codebook_f64(double levels[16]) {
   for (int i = 0; i < 16; ++i) levels[i] = v[i] / mx;
 }
 
+void thresholds_f32(const float levels[16], float thresholds[15]) {
+  for (int i = 0; i < 15; ++i) {
+    // exact midpoint of two float32 values in float64, then the smallest float32 above it
+    const double m = (static_cast<double>(levels[i]) + static_cast<double>(levels[i + 1])) * 0.5;
+    float t = static_cast<float>(m);
+    if (static_cast<double>(t) <= m) t = std::nextafter(t, INFINITY);
+    thresholds[i] = t;
+  }
+  // Of two equal levels the upper one is never the nearest (ties go to the lower
+  // index): its threshold moves up to the next one, so the count skips it.
+  for (int i = 13; i >= 0; --i)
+    if (levels[i] == levels[i + 1]) thresholds[i] = thresholds[i + 1];
+}
+
 void build_codebook_f32(float levels[16], float thresholds[15]) {
   double l64[16];
   build_codebook_f64(l64);
   float l32[16];
   for (int i = 0; i < 16; ++i) l32[i] = static_cast<float>(l64[i]);
   if (levels) std::memcpy(levels, l32, sizeof(l32));
-  if (thresholds) {
-    for (int i = 0; i < 15; ++i) {
-      // exact midpoint of two float32 values in float64, then the smallest float32 above it
-      const double m = (static_cast<double>(l32[i]) + static_cast<double>(l32[i + 1])) * 0.5;
-      float t = static_cast<float>(m);
-      if (static_cast<double>(t) <= m) t = std::nextafter(t, INFINITY);
-      thresholds[i] = t;
+  if (thresholds) thresholds_f32(l32, thresholds);
+}
+
+bool build_format_codebook_f32(int codebook, float levels[16], float thresholds[15]) {
+  float l32[16];
+  if (codebook == QLORA_CB_NF4) {
+    build_codebook_f32(l32, nullptr);
+  } else if (codebook == QLORA_CB_INT4) {
+    // the symmetric absmax integer grid k/7, k = -7..7, plus -8/7 (never the nearest in [-1, 1])
+    for (int i = 0; i < 16; ++i) l32[i] = static_cast<float>((i - 8) / 7.0);
+  } else if (codebook == QLORA_CB_FP4_E2M1 || codebook == QLORA_CB_FP4_E3M0) {
+    // non-negative values of the sign + 3-bit float layout, divided by the largest;
+    // both zeros of the layout are the level +0
+    static const double e2m1[8] = {0, 0.5, 1, 1.5, 2, 3, 4, 6};
+    static const double e3m0[8] = {0, 0.25, 0.5, 1, 2, 4, 8, 16};
+    const double *pos = codebook == QLORA_CB_FP4_E2M1 ? e2m1 : e3m0;
+    for (int i = 1; i < 8; ++i) {
+      l32[8 + i] = static_cast<float>(pos[i] / pos[7]);
+      l32[7 - i] = -l32[8 + i];
     }
+    l32[7] = 0.0f;
+    l32[8] = 0.0f;
+  } else {
+    return false;
   }
+  if (levels) std::memcpy(levels, l32, sizeof(l32));
+  if (thresholds) thresholds_f32(l32, thresholds);
+  return true;
 }
 
 }  // namespace qlora

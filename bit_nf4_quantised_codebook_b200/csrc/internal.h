@@ -23,6 +23,8 @@ const TimingHooks &timing_hooks();
 // Host code-book construction (codebook.cpp).
 void build_codebook_f64(double levels[16]);
 void build_codebook_f32(float levels[16], float thresholds[15]);
+void thresholds_f32(const float levels[16], float thresholds[15]);
+bool build_format_codebook_f32(int codebook, float levels[16], float thresholds[15]);
 
 cudaError_t launch_quantize(const uint16_t *W, int64_t nb, uint8_t *codes, uint8_t *c2q, float *c1, float *mean,
                             float *ws_absmax, double *ws_gsum, int64_t gsum_size, const Nf4Thresholds &thr,
@@ -31,6 +33,7 @@ cudaError_t launch_quantize(const uint16_t *W, int64_t nb, uint8_t *codes, uint8
 // sums (launch_group_sums, when the caller has not formed them), the fixed-order
 // mean, then the E4M3 codes and group scales.
 cudaError_t launch_group_sums(const float *ws_absmax, int64_t nb, double *ws_gsum, cudaStream_t st);
+cudaError_t launch_mean_tree(double *ws_gsum, int64_t nb, int64_t gsum_size, float *mean, cudaStream_t st);
 cudaError_t launch_mean_and_double_quant(const float *ws_absmax, int64_t nb, double *ws_gsum, int64_t gsum_size,
                                          float *mean, uint8_t *c2q, float *c1, cudaStream_t st);
 cudaError_t launch_dequantize(const uint8_t *codes, const uint8_t *c2q, const float *c1, const float *mean,
@@ -42,6 +45,15 @@ cudaError_t launch_merge_requantize(const qlora_nf4_weight &w, const uint16_t *A
                                     double *ws_gsum, int64_t gsum_size, const Nf4Levels &lv,
                                     const Nf4Thresholds &thr, int *dev_err, unsigned long long timeout_ns,
                                     cudaStream_t st);
+// formats.cu
+cudaError_t launch_quantize_format(const uint16_t *W, const qlora_qweight &w, const float levels[16],
+                                   const float thresholds[15], float *ws_absmax, double *ws_gsum, int64_t gsum_size,
+                                   int *dev_err, cudaStream_t st);
+cudaError_t launch_dequantize_format(const qlora_qweight &w, const float levels[16], uint16_t *out, cudaStream_t st);
+cudaError_t launch_quant_error(const uint16_t *W, const uint16_t *W_hat, int64_t n, double *stats, int num_sms,
+                               cudaStream_t st);
+cudaError_t launch_double_quant_int8(const float *ws_absmax, int64_t nb, const float *mean, int8_t *c2q, float *c1,
+                                     cudaStream_t st);
 // adamw.cu
 using AdamwTensor = qlora_adamw_tensor;
 constexpr int kAdamwMaxTensors = QLORA_ADAMW_MAX_TENSORS;

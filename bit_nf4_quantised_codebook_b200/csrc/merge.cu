@@ -9,18 +9,20 @@
 // and W_eff is quantised exactly as the quantiser does it (64-element absmax
 // blocks, NF4 codes, then the double quantisation of the block constants).
 //
-// k_merge_quant, one CTA of 128 threads per 128 (W rows n) x 128 (columns k) tile:
+// k_merge_quant: persistent CTAs of 128 threads; a tile is 128 rows n x 64
+// columns k (one 64-weight block per row), so thread = TMEM lane = W row = one block:
 //   - thread 0 loads the tile's slices of B (MN-major: n contiguous) and A
 //     (K-major: j contiguous) by TMA, then issues rpad/16 tcgen05 MMAs
-//     (M = 128 rows n, N = 128 columns k, K = 16) into a 128-column TMEM
+//     (M = 128 rows n, N = 64 columns k, K = 16) into a 64-column TMEM
 //     accumulator: sum_j B[j, n]·A[k, j] in float32 (rpad = r rounded up to 16;
 //     rows of B and columns of A beyond r arrive as zeros);
-//   - meanwhile each thread loads the old codes and block constants of its
-//     row's two 64-element blocks (thread = TMEM lane = W row);
-//   - each thread then reads its row's accumulator columns 32 at a time,
-//     decodes ŵ with the block's lookup table, forms the merged bfloat16 values
-//     and codes the block: absmax, exact quotient, nearest level by the bucket
-//     table, nibble packing — the quantiser's own steps (nf4_quant.cuh).
+//   - as soon as those MMAs complete it loads the next tile's slices into the
+//     same shared memory, and every thread loads the old codes and block
+//     constant of its next block, so both are in flight during the epilogue;
+//   - the epilogue reads the row's accumulator 32 columns at a time, decodes ŵ
+//     with the block's lookup table, forms the merged bfloat16 values and codes
+//     the block: absmax, exact quotient, nearest level by the bucket table,
+//     nibble packing — the quantiser's own steps (nf4_quant.cuh).
 // The float32 absmax of every block goes to the workspace; the group sums, the
 // fixed-order mean and the E4M3 codes follow in quantize.cu's kernels.
 //
@@ -43,11 +45,13 @@
 namespace qlora {
 namespace {
 
-constexpr int kTile = 128;                     // rows n and columns k per CTA
-constexpr uint32_t kChunkBytes = 16384;        // one 64-wide slice of r: 128 rows x 128 B
+constexpr int kRows = 128;                     // rows n per tile (MMA M)
+constexpr int kCols = 64;                      // columns k per tile (MMA N): one block per row
+constexpr uint32_t kBSlice = 16384;            // B: 64 of r x 128 rows n (two 64-wide boxes)
+constexpr uint32_t kASlice = 8192;             // A: 64 rows k x 64 of r
 constexpr uint32_t kTabBytes = kBuckets * 32 * sizeof(CodeBucket);
 constexpr unsigned long long kMergeDrainNs = 1000000000ull;
-constexpr uint32_t kIdesc = idesc_bf16(kTile, kTile, true, false);  // A operand (B's slice) MN-major
+constexpr uint32_t kIdesc = idesc_bf16(kRows, kCols, true, false);  // A operand (B's slice) MN-major
 static_assert(kTabBytes == 16384, "bucket table is 16 KiB");
 
 struct MergeArgs {
@@ -70,25 +74,50 @@ struct MergeArgs {
 
 __device__ __forceinline__ uint4 ld_v4(const void *p) { return *reinterpret_cast<const uint4 *>(p); }
 
-__global__ void __launch_bounds__(128) k_merge_quant(const __grid_constant__ CUtensorMap map_b,
-                                                      const __grid_constant__ CUtensorMap map_a,
-                                                      const __grid_constant__ MergeArgs p) {
+// The old codes and block constant of one block (row n, 64-column block kb).
+struct BlockIn {
+  uint32_t words[8];
+  float c2h;
+  bool valid;
+};
+
+__device__ __forceinline__ void load_block(const MergeArgs &p, int64_t tile, int64_t tiles, int row, float mu,
+                                           BlockIn &in) {
+  const int64_t kblocks = p.K / kCols;
+  const int64_t n = (tile / kblocks) * kRows + row;
+  in.valid = tile < tiles && n < p.N;
+  in.c2h = 0.f;
+#pragma unroll
+  for (int i = 0; i < 8; ++i) in.words[i] = 0x77777777u;
+  if (in.valid) {
+    const int64_t b = n * kblocks + tile % kblocks;
+    const uint4 q0 = ld_v4(p.codes_in + b * 32), q1 = ld_v4(p.codes_in + b * 32 + 16);
+    in.words[0] = q0.x, in.words[1] = q0.y, in.words[2] = q0.z, in.words[3] = q0.w;
+    in.words[4] = q1.x, in.words[5] = q1.y, in.words[6] = q1.z, in.words[7] = q1.w;
+    in.c2h = reconstruct_c2(p.c2q_in[b], p.c1_in[b >> 8], mu);
+  }
+}
+
+__global__ void __launch_bounds__(128, 4) k_merge_quant(const __grid_constant__ CUtensorMap map_b,
+                                                         const __grid_constant__ CUtensorMap map_a,
+                                                         const __grid_constant__ MergeArgs p) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  uint8_t *sB = smem;                               // nch x (two 64-row halves of n, 8 KiB each)
-  uint8_t *sA = smem + p.nch * kChunkBytes;         // nch x 128 rows k x 128 B
-  CodeBucket(*s_tab)[32] = reinterpret_cast<CodeBucket(*)[32]>(smem + 2 * p.nch * kChunkBytes);
+  uint8_t *sB = smem;                          // nch x (two 64-row halves of n, 8 KiB each)
+  uint8_t *sA = smem + p.nch * kBSlice;        // nch x 64 rows k x 128 B
+  CodeBucket(*s_tab)[32] = reinterpret_cast<CodeBucket(*)[32]>(smem + p.nch * (kBSlice + kASlice));
+  __shared__ CodeBucket s_bucket[kBuckets];
   __shared__ uint64_t tma_bar, mma_bar;
   __shared__ uint32_t tmem_slot;
   __shared__ volatile int abort_flag;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int64_t tiles_k = (p.K + kTile - 1) / kTile;
-  const int64_t n0 = (static_cast<int64_t>(blockIdx.x) / tiles_k) * kTile;
-  const int64_t k0 = (static_cast<int64_t>(blockIdx.x) % tiles_k) * kTile;
+  const int row = 32 * warp + lane;
+  const int64_t kblocks = p.K / kCols;
+  const int64_t tiles = ((p.N + kRows - 1) / kRows) * kblocks;
 
   if (warp == 0) {
-    tmem_alloc(&tmem_slot, kTile);
+    tmem_alloc(&tmem_slot, kCols);
     tmem_relinquish();
   }
   if (threadIdx.x == 32) {
@@ -99,95 +128,90 @@ __global__ void __launch_bounds__(128) k_merge_quant(const __grid_constant__ CUt
     tma_prefetch_desc(&map_b);
     tma_prefetch_desc(&map_a);
   }
-  for (int i = threadIdx.x; i < kBuckets * 32; i += blockDim.x) s_tab[i >> 5][i & 31] = make_bucket(i >> 5, p.thr.t);
+  // bucket table: 64 entries, then one copy per lane (conflict-free lookups)
+  if (threadIdx.x < kBuckets) s_bucket[threadIdx.x] = make_bucket(threadIdx.x, p.thr.t);
+  __syncthreads();
+  for (int i = threadIdx.x; i < kBuckets * 32; i += blockDim.x) s_tab[i >> 5][i & 31] = s_bucket[i >> 5];
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = tmem_slot;
+  const uint32_t trow = tmem + (static_cast<uint32_t>(32 * warp) << 16);
 
   pdl_wait();
   pdl_launch_dependents();
 
-  if (threadIdx.x == 0) {
-    mbar_arrive_expect_tx(&tma_bar, static_cast<uint32_t>(p.nch) * 2 * kChunkBytes);
+  auto issue_loads = [&](int64_t tile) {
+    const int n0 = static_cast<int>((tile / kblocks) * kRows), k0 = static_cast<int>((tile % kblocks) * kCols);
+    mbar_arrive_expect_tx(&tma_bar, static_cast<uint32_t>(p.nch) * (kBSlice + kASlice));
     for (int c = 0; c < p.nch; ++c) {
-      tma_load_2d(sB + c * kChunkBytes, &map_b, &tma_bar, static_cast<int>(n0), 64 * c);
-      tma_load_2d(sB + c * kChunkBytes + kChunkBytes / 2, &map_b, &tma_bar, static_cast<int>(n0) + 64, 64 * c);
-      tma_load_2d(sA + c * kChunkBytes, &map_a, &tma_bar, 64 * c, static_cast<int>(k0));
+      tma_load_2d(sB + c * kBSlice, &map_b, &tma_bar, n0, 64 * c);
+      tma_load_2d(sB + c * kBSlice + kBSlice / 2, &map_b, &tma_bar, n0 + 64, 64 * c);
+      tma_load_2d(sA + c * kASlice, &map_a, &tma_bar, 64 * c, k0);
     }
-  }
+  };
 
-  // The old codes and constants of this thread's two blocks (row n, 64-column blocks kb0, kb0 + 1).
-  const int64_t n = n0 + 32 * warp + lane;
-  const int64_t kblocks = p.K / 64;
-  const int64_t kb0 = k0 / 64;
-  bool valid[2];
-  uint32_t words[2][8];
-  float c2h[2];
   const float mu = *p.mean_in;
-#pragma unroll
-  for (int bb = 0; bb < 2; ++bb) {
-    valid[bb] = n < p.N && kb0 + bb < kblocks;
-    c2h[bb] = 0.f;
-    if (valid[bb]) {
-      const int64_t b = n * kblocks + kb0 + bb;
-      const uint4 q0 = ld_v4(p.codes_in + b * 32), q1 = ld_v4(p.codes_in + b * 32 + 16);
-      words[bb][0] = q0.x, words[bb][1] = q0.y, words[bb][2] = q0.z, words[bb][3] = q0.w;
-      words[bb][4] = q1.x, words[bb][5] = q1.y, words[bb][6] = q1.z, words[bb][7] = q1.w;
-      c2h[bb] = reconstruct_c2(p.c2q_in[b], p.c1_in[b >> 8], mu);
-    } else {
-#pragma unroll
-      for (int i = 0; i < 8; ++i) words[bb][i] = 0x77777777u;
-    }
+  int64_t tile = blockIdx.x;
+  int pending_tma = -1, pending_mma = -1;  // (thread 0) parity of an issued, not yet awaited, phase
+  if (threadIdx.x == 0 && tile < tiles) {
+    issue_loads(tile);
+    pending_tma = 0;
   }
-
-  bool issued = false, mma_issued = false;
-  if (threadIdx.x == 0) {
-    issued = true;
-    if (mbar_wait_bounded(&tma_bar, 0, &abort_flag, p.dev_err, p.timeout_ns)) {
+  BlockIn cur;
+  load_block(p, tile, tiles, row, mu, cur);
+  bool bad = false;
+  for (uint32_t it = 0; tile < tiles; tile += gridDim.x, ++it) {
+    const uint32_t ph = it & 1;
+    if (threadIdx.x == 0 && mbar_wait_bounded(&tma_bar, ph, &abort_flag, p.dev_err, p.timeout_ns)) {
+      pending_tma = -1;
       tc_fence_after();
       const uint32_t a_base = smem_u32(sB), b_base = smem_u32(sA);
       for (int kk = 0; kk < p.ksteps; ++kk) {
-        const uint32_t off = static_cast<uint32_t>(kk >> 2) * kChunkBytes;
-        const uint64_t ad = smem_desc_sw128(a_base + off + (kk & 3) * 2048, kChunkBytes / 2, 1024);
-        const uint64_t bd = smem_desc_sw128(b_base + off + (kk & 3) * 32, 16, 1024);
+        const uint64_t ad = smem_desc_sw128(a_base + (kk >> 2) * kBSlice + (kk & 3) * 2048, kBSlice / 2, 1024);
+        const uint64_t bd = smem_desc_sw128(b_base + (kk >> 2) * kASlice + (kk & 3) * 32, 16, 1024);
         mma_bf16_ss(tmem, ad, bd, kIdesc, kk > 0 ? 1u : 0u);
       }
       mma_commit(&mma_bar);
-      mma_issued = true;
+      pending_mma = static_cast<int>(ph);
     }
-  }
+    const bool ok = mbar_wait_bounded(&mma_bar, ph, &abort_flag, p.dev_err, p.timeout_ns);
+    if (__syncthreads_or(!ok)) break;  // the same decision in every thread
+    tc_fence_after();
+    const int64_t next = tile + gridDim.x;
+    if (threadIdx.x == 0) {
+      pending_mma = -1;
+      if (next < tiles) {  // the MMAs are done with the shared slices: refill them now
+        issue_loads(next);
+        pending_tma = static_cast<int>((it + 1) & 1);
+      }
+    }
+    BlockIn nxt;
+    load_block(p, next, tiles, row, mu, nxt);
 
-  bool ok = mbar_wait_bounded(&mma_bar, 0, &abort_flag, p.dev_err, p.timeout_ns);
-  ok = __all_sync(0xFFFFFFFFu, ok);  // the accumulator loads below are warp-wide
-  tc_fence_after();
-  bool bad = false;
-  if (ok) {
-    const uint32_t trow = tmem + (static_cast<uint32_t>(32 * warp) << 16);
+    const BlockLut lut = make_lut(cur.c2h, p.lv);
+    uint32_t merged[32];  // bf16x2 words of W_eff, element 2i in the low half of word i
 #pragma unroll
-    for (int bb = 0; bb < 2; ++bb) {
-      const BlockLut lut = make_lut(c2h[bb], p.lv);
-      uint32_t merged[32];  // bf16x2 words of W_eff, element 2i in the low half of word i
+    for (int half = 0; half < 2; ++half) {
+      uint32_t acc[32];
+      tmem_ld32(trow + 32 * half, acc);
+      tmem_ld_wait();
 #pragma unroll
-      for (int half = 0; half < 2; ++half) {
-        uint32_t acc[32];
-        tmem_ld32(trow + 64 * bb + 32 * half, acc);
-        tmem_ld_wait();
+      for (int c = 0; c < 4; ++c) {
+        uint32_t o[4];
+        decode8(cur.words[4 * half + c], lut, o);
 #pragma unroll
-        for (int c = 0; c < 4; ++c) {
-          uint32_t o[4];
-          decode8(words[bb][4 * half + c], lut, o);
-#pragma unroll
-          for (int q = 0; q < 4; ++q) {
-            const int e = 8 * c + 2 * q;  // element within this half
-            const float w0 = __uint_as_float(o[q] << 16), w1 = __uint_as_float(o[q] & 0xFFFF0000u);
-            const float m0 = __fmaf_rn(p.s, __uint_as_float(acc[e]), w0);
-            const float m1 = __fmaf_rn(p.s, __uint_as_float(acc[e + 1]), w1);
-            merged[16 * half + 4 * c + q] = pack_bf16x2(m0, m1);
-          }
+        for (int q = 0; q < 4; ++q) {
+          const int e = 8 * c + 2 * q;  // element within this half
+          const float w0 = __uint_as_float(o[q] << 16), w1 = __uint_as_float(o[q] & 0xFFFF0000u);
+          const float m0 = __fmaf_rn(p.s, __uint_as_float(acc[e]), w0);
+          const float m1 = __fmaf_rn(p.s, __uint_as_float(acc[e + 1]), w1);
+          merged[16 * half + 4 * c + q] = pack_bf16x2(m0, m1);
         }
       }
-      if (!valid[bb]) continue;
+    }
+    tc_fence_before();
+    if (cur.valid) {
       float amax = 0.f;
 #pragma unroll
       for (int i = 0; i < 32; ++i) {
@@ -227,32 +251,36 @@ __global__ void __launch_bounds__(128) k_merge_quant(const __grid_constant__ CUt
 #pragma unroll
         for (int c = 0; c < 8; ++c) packed[c] = 0x77777777u;  // all-zero block: the zero level
       }
-      const int64_t b = n * kblocks + kb0 + bb;
+      const int64_t n = (tile / kblocks) * kRows + row, kb = tile % kblocks;
+      const int64_t b = n * kblocks + kb;
       uint4 *cp = reinterpret_cast<uint4 *>(p.codes_out + b * 32);
       cp[0] = make_uint4(packed[0], packed[1], packed[2], packed[3]);
       cp[1] = make_uint4(packed[4], packed[5], packed[6], packed[7]);
       p.absmax[b] = amax;
       if (p.w_merged) {
-        uint4 *wp = reinterpret_cast<uint4 *>(p.w_merged + n * p.K + (kb0 + bb) * 64);
+        uint4 *wp = reinterpret_cast<uint4 *>(p.w_merged + n * p.K + kb * kCols);
 #pragma unroll
         for (int i = 0; i < 8; ++i)
           wp[i] = make_uint4(merged[4 * i], merged[4 * i + 1], merged[4 * i + 2], merged[4 * i + 3]);
       }
     }
+    __syncthreads();  // every row has read the accumulator: the next MMAs may overwrite it
+    tc_fence_after();
+    cur = nxt;
   }
   if (bad && p.dev_err) atomicOr(p.dev_err, QLORA_DEVERR_NONFINITE);
 
-  if (issued && abort_flag) {
-    // a wait gave up: the copies (and MMAs) issued must land before TMEM and shared memory go away
+  if (threadIdx.x == 0 && (pending_tma >= 0 || pending_mma >= 0)) {
+    // a wait gave up: what was issued must land before TMEM and shared memory go away
     int dummy = 0;
-    mbar_wait_bounded(&tma_bar, 0, &dummy, nullptr, kMergeDrainNs);
-    if (mma_issued) mbar_wait_bounded(&mma_bar, 0, &dummy, nullptr, kMergeDrainNs);
+    if (pending_tma >= 0) mbar_wait_bounded(&tma_bar, static_cast<uint32_t>(pending_tma), &dummy, nullptr, kMergeDrainNs);
+    if (pending_mma >= 0) mbar_wait_bounded(&mma_bar, static_cast<uint32_t>(pending_mma), &dummy, nullptr, kMergeDrainNs);
   }
   tc_fence_before();
   __syncthreads();
   if (warp == 0) {
     tc_fence_after();
-    tmem_dealloc(tmem, kTile);
+    tmem_dealloc(tmem, kCols);
   }
 }
 
@@ -260,7 +288,7 @@ __global__ void __launch_bounds__(128) k_merge_quant(const __grid_constant__ CUt
 
 size_t merge_smem_bytes(int r) {
   const int nch = (r + 63) / 64;
-  return 2 * static_cast<size_t>(nch) * kChunkBytes + kTabBytes + 1024;
+  return static_cast<size_t>(nch) * (kBSlice + kASlice) + kTabBytes + 1024;
 }
 
 cudaError_t launch_merge_requantize(const qlora_nf4_weight &w, const uint16_t *A, const uint16_t *B, int r, float s,
@@ -269,8 +297,8 @@ cudaError_t launch_merge_requantize(const qlora_nf4_weight &w, const uint16_t *A
                                     const Nf4Thresholds &thr, int *dev_err, unsigned long long timeout_ns,
                                     cudaStream_t st) {
   CUtensorMap mb, ma;
-  // B [r, N] read MN-major (box 64 n x 64 j); A [K, r] read K-major (box 64 j x 128 k)
-  if (!map_bf16_mn(&mb, B, w.N, r) || !map_bf16_kmajor(&ma, A, r, w.K, kTile)) return cudaErrorInvalidValue;
+  // B [r, N] read MN-major (box 64 n x 64 j); A [K, r] read K-major (box 64 j x 64 k)
+  if (!map_bf16_mn(&mb, B, w.N, r) || !map_bf16_kmajor(&ma, A, r, w.K, kCols)) return cudaErrorInvalidValue;
   MergeArgs a;
   a.codes_in = w.codes;
   a.c2q_in = w.c2q;
@@ -289,17 +317,23 @@ cudaError_t launch_merge_requantize(const qlora_nf4_weight &w, const uint16_t *A
   a.dev_err = dev_err;
   a.timeout_ns = timeout_ns;
   const size_t smem = merge_smem_bytes(r);
-  // At most 4 CTAs fit on an SM by shared memory (>= 48 KiB each), so their
-  // 128-column TMEM allocations (512 columns per SM) never wait on one another.
-  static_assert(2 * kChunkBytes + kTabBytes >= 48 * 1024, "at most 4 CTAs per SM");
+  // At most 5 CTAs fit on an SM by shared memory (>= 40 KiB each), so their
+  // 64-column TMEM allocations (512 columns per SM) never wait on one another.
+  static_assert(kBSlice + kASlice + kTabBytes >= 40 * 1024, "at most 5 CTAs per SM");
   cudaError_t e = cudaFuncSetAttribute(k_merge_quant, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        static_cast<int>(smem));
   if (e != cudaSuccess) return e;
-  const int64_t tiles = ((w.N + kTile - 1) / kTile) * ((w.K + kTile - 1) / kTile);
-  if (tiles > 0x7FFFFFFF) return cudaErrorInvalidValue;
+  int per_sm = 0;
+  e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, k_merge_quant, 128, smem);
+  if (e != cudaSuccess) return e;
+  int dev = 0, sms = 148;
+  if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  const int64_t tiles = ((w.N + kRows - 1) / kRows) * (w.K / kCols);
+  const int64_t slots = static_cast<int64_t>(per_sm > 0 ? per_sm : 1) * sms;
+  const int64_t grid = tiles < slots ? tiles : slots;
   const TimingHooks &hk = timing_hooks();
   if (hk.fwd_begin) cudaEventRecord(hk.fwd_begin, st);
-  e = launch_k(k_merge_quant, dim3(static_cast<unsigned>(tiles)), dim3(128), smem, st, 1, mb, ma, a);
+  e = launch_k(k_merge_quant, dim3(static_cast<unsigned>(grid)), dim3(128), smem, st, 1, mb, ma, a);
   if (e != cudaSuccess) return e;
   if (hk.fwd_end) cudaEventRecord(hk.fwd_end, st);
   const int64_t nb = w.N * w.K / 64;

@@ -261,10 +261,15 @@ cudaError_t launch_quantize(const uint16_t *W, int64_t nb, uint8_t *codes, uint8
   return launch_mean_and_double_quant(ws_absmax, nb, ws_gsum, gsum_size, mean, c2q, c1, st);
 }
 
+cudaError_t launch_mean_tree(double *ws_gsum, int64_t nb, int64_t gsum_size, float *mean, cudaStream_t st) {
+  const int64_t ng = (nb + 255) / 256;
+  return launch_k(k_mean_tree, dim3(1), dim3(1024), 0, st, 1, ws_gsum, ng, gsum_size, nb, mean);
+}
+
 cudaError_t launch_mean_and_double_quant(const float *ws_absmax, int64_t nb, double *ws_gsum, int64_t gsum_size,
                                          float *mean, uint8_t *c2q, float *c1, cudaStream_t st) {
   const int64_t ng = (nb + 255) / 256;
-  cudaError_t e = launch_k(k_mean_tree, dim3(1), dim3(1024), 0, st, 1, ws_gsum, ng, gsum_size, nb, mean);
+  cudaError_t e = launch_mean_tree(ws_gsum, nb, gsum_size, mean, st);
   if (e != cudaSuccess) return e;
   return launch_k(k_double_quant, dim3(static_cast<unsigned>(ng)), dim3(256), 0, st, 1, ws_absmax, nb,
                   static_cast<const float *>(mean), c2q, c1);

@@ -261,6 +261,89 @@ qlora_status qlora_adamw_step(const qlora_adamw_tensor *tensors, int count, floa
  */
 qlora_status qlora_selftest_bounded_wait(unsigned timeout_us, int *dev_err, int *gave_up, void *stream);
 
+/*
+ * Storage-format variants, for the quantisation study that sets NF4 against
+ * other 4-bit types, block sizes and treatments of the block constants
+ * ("QLoRA: Efficient Finetuning of Quantized LLMs", intuitivepapers.ai:
+ * §Quantize in blocks, §NormalFloat — the uniform Int4 grid —, §Double
+ * quantization, §It matches 16-bit finetuning — "4-bit float variants";
+ * "QLoRA Review", tildalice.io, §What Would Trip You Up in Practice — block
+ * size trades precision against overhead).  The linear layer itself always
+ * uses NF4, blocks of 64 and E4M3 constants (qlora_nf4_weight above).
+ *
+ * Code books (16 ascending float32 levels in [-1, 1]):
+ *   QLORA_CB_NF4       the NF4 levels of qlora_build_codebook;
+ *   QLORA_CB_INT4      k/7 for k = -8..7 (the symmetric absmax integer grid;
+ *                      -8/7 is never the nearest level of a value in [-1, 1]);
+ *   QLORA_CB_FP4_E2M1  +-{0, 0.5, 1, 1.5, 2, 3, 4, 6} / 6;
+ *   QLORA_CB_FP4_E3M0  +-{0, 0.25, 0.5, 1, 2, 4, 8, 16} / 16
+ *                      (the float layouts' +0 and -0 are both the level +0).
+ * Block sizes 32, 64, 128, 256 (consecutive weights along K; K % block == 0).
+ * Block constants (absmax c of each block):
+ *   QLORA_DQ_NONE  stored as float32;
+ *   QLORA_DQ_E4M3  the second quantisation of qlora_quantize (mean, groups of
+ *                  256 blocks, E4M3 codes of the centred constants);
+ *   QLORA_DQ_INT8  the same with the int8 absmax grid: S_g = float32(amax_g/127),
+ *                  e = round-half-even(float32(dev/S_g)), reconstruction
+ *                  fmaf(e, S_g, mu).
+ * Codes: x = float32(w / c), nearest level, ties to the lower index (of two
+ * equal levels the first); an all-zero block codes to the first zero level.
+ */
+enum { QLORA_CB_NF4 = 0, QLORA_CB_INT4 = 1, QLORA_CB_FP4_E2M1 = 2, QLORA_CB_FP4_E3M0 = 3 };
+enum { QLORA_DQ_NONE = 0, QLORA_DQ_E4M3 = 1, QLORA_DQ_INT8 = 2 };
+
+typedef struct qlora_format {
+  int codebook;  /* QLORA_CB_* */
+  int block;     /* 32, 64, 128 or 256 */
+  int dq;        /* QLORA_DQ_* */
+} qlora_format;
+
+typedef struct qlora_qweight {
+  int64_t N, K;
+  qlora_format fmt;
+  uint8_t *codes;  /* N*K/2 bytes, two codes per byte (even element in the high nibble) */
+  void *consts;    /* per block: float32 c (DQ_NONE) or one byte (E4M3 code / int8) */
+  float *c1;       /* per group of 256 blocks (DQ_E4M3, DQ_INT8; else unused, may be NULL) */
+  float *mean;     /* 1 float (DQ_E4M3, DQ_INT8; else unused, may be NULL) */
+} qlora_qweight;
+
+/* Levels and thresholds of a code book (host); thresholds as in
+ * qlora_build_codebook, with the threshold of the upper of two equal levels
+ * raised to the next one.  QLORA_ERR_INVALID_ARG for an unknown code book. */
+qlora_status qlora_format_codebook(int codebook, float levels[16], float thresholds[15]);
+
+/* Byte sizes of codes, consts and c1 for a format and shape. */
+qlora_status qlora_format_sizes(const qlora_format *fmt, int64_t N, int64_t K, size_t *codes_bytes,
+                                size_t *consts_bytes, size_t *c1_bytes);
+
+/* Workspace bytes of qlora_quantize_format for a format and shape. */
+qlora_status qlora_format_workspace_size(const qlora_format *fmt, int64_t N, int64_t K, size_t *bytes);
+
+/*
+ * qlora_quantize_format — W (device, N x K bfloat16) into w's buffers in the
+ * format w->fmt.  ws: qlora_format_workspace_size() bytes (16-byte aligned).
+ * The mean and group sums follow qlora_quantize's fixed order.  A non-finite
+ * weight sets QLORA_DEVERR_NONFINITE.  Deterministic.  All device pointers
+ * 16-byte aligned.  Errors: QLORA_ERR_INVALID_ARG (null pointer, unknown code
+ * book or constant mode), QLORA_ERR_UNSUPPORTED_SHAPE (block not 32/64/128/256,
+ * K % block != 0), QLORA_ERR_MISALIGNED, QLORA_ERR_WORKSPACE.
+ */
+qlora_status qlora_quantize_format(const uint16_t *W, const qlora_qweight *w, void *ws, size_t ws_bytes,
+                                   int *dev_err, void *stream);
+
+/* w_hat = bf16_rn(float32(level[code] * c_hat)) for every weight, into W_out
+ * (device, N x K bfloat16); c_hat = c, or the reconstructed constant. */
+qlora_status qlora_dequantize_format(const qlora_qweight *w, uint16_t *W_out, void *stream);
+
+/*
+ * qlora_quant_error — error of a round trip, for the study's curves.
+ * W, W_hat: device, n bfloat16 each (16-byte aligned).  stats: device,
+ * 3 doubles (8-byte aligned), overwritten:
+ * stats[0] = sum (w - w_hat)^2, stats[1] = sum w^2, stats[2] = max |w - w_hat|
+ * (sums in float64; their order is unspecified).
+ */
+qlora_status qlora_quant_error(const uint16_t *W, const uint16_t *W_hat, int64_t n, double *stats, void *stream);
+
 /* Number of kernels this library has launched in this process so far. */
 uint64_t qlora_kernel_launch_count(void);
 

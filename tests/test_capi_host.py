@@ -110,6 +110,56 @@ def test_merge_validation(api):
     assert call(wm=8192 - 16) == 1                                        # W_merged over w's buffers
 
 
+def test_format_code_books_match_oracle(api):
+    """Levels bit-exact; thresholds give the oracle's nearest level (ties to the
+    lower index, the upper of two equal levels never chosen)."""
+    from oracle import formats, nf4
+    rng = np.random.default_rng(3)
+    for cb in formats.CODEBOOKS:
+        lv, th = api.qlora_format_codebook(cb)
+        lv = np.array(lv, np.float32)
+        th = np.array(th, np.float32)
+        ref = formats.codebook(cb)
+        assert np.array_equal(lv.view(np.uint32), ref.view(np.uint32)), cb
+        assert np.all(np.diff(th) >= 0), cb
+        m = (ref[:-1].astype(np.float64) + ref[1:].astype(np.float64)) / 2
+        x = np.concatenate([rng.uniform(-1, 1, 50000), m[np.abs(m) <= 1], [0.0, -1.0, 1.0, 1e-30, -1e-30]])
+        x = x.astype(np.float32)
+        x = np.concatenate([x, np.nextafter(x, np.float32(2)), np.nextafter(x, np.float32(-2))])
+        x = x[np.abs(x) <= 1]
+        codes = np.searchsorted(th, x, side="right")          # #{i : x >= t_i}
+        assert np.array_equal(codes, nf4.nearest_level(x, ref)), cb
+    assert api.lib().qlora_format_codebook(4, None, None) == 1
+
+
+def test_format_validation(api):
+    L = api.lib()
+    F, Q = api._Format, api._QWeight
+    n = ctypes.c_size_t()
+    assert L.qlora_format_sizes(ctypes.byref(F(0, 48, 1)), 16, 96, None, None, None) == 2      # block
+    assert L.qlora_format_sizes(ctypes.byref(F(4, 64, 1)), 16, 128, None, None, None) == 1     # code book
+    assert L.qlora_format_sizes(ctypes.byref(F(0, 64, 3)), 16, 128, None, None, None) == 1     # constants
+    assert L.qlora_format_sizes(ctypes.byref(F(0, 128, 1)), 16, 192, None, None, None) == 2    # K % block
+    a, b, c = ctypes.c_size_t(), ctypes.c_size_t(), ctypes.c_size_t()
+    assert L.qlora_format_sizes(ctypes.byref(F(2, 32, 0)), 16, 128, ctypes.byref(a), ctypes.byref(b),
+                                ctypes.byref(c)) == 0
+    assert (a.value, b.value, c.value) == (1024, 64 * 4, 0)
+    assert L.qlora_format_sizes(ctypes.byref(F(1, 256, 2)), 16, 4096, ctypes.byref(a), ctypes.byref(b),
+                                ctypes.byref(c)) == 0
+    assert (a.value, b.value, c.value) == (32768, 256, 4)
+    assert L.qlora_format_workspace_size(ctypes.byref(F(0, 32, 1)), 16, 128, ctypes.byref(n)) == 0 and n.value > 0
+    w = Q(16, 128, F(0, 64, 1), 4096, 8192, 12288, 16384)
+    assert L.qlora_quantize_format(None, ctypes.byref(w), 1 << 20, 1 << 20, None, None) == 1
+    assert L.qlora_quantize_format(17 * 16 + 1, ctypes.byref(w), 1 << 20, 1 << 20, None, None) == 3
+    assert L.qlora_quantize_format(1 << 21, ctypes.byref(Q(16, 128, F(0, 64, 1), 4096, 8192, 0, 16384)),
+                                   1 << 20, 1 << 20, None, None) == 1                         # c1 needed
+    assert L.qlora_quantize_format(1 << 21, ctypes.byref(w), 1 << 20, 8, None, None) == 5     # workspace
+    assert L.qlora_dequantize_format(ctypes.byref(Q(16, 100, F(0, 64, 0), 4096, 8192, 0, 0)), 1 << 21, None) == 2
+    assert L.qlora_quant_error(None, 16, 8, 16, None) == 1
+    assert L.qlora_quant_error(16, 16, 0, 16, None) == 1
+    assert L.qlora_quant_error(16, 16, 8, 12, None) == 3
+
+
 def test_product_path_has_no_cpu_fallback():
     """The binding never imports the oracle; the package refuses to run without the library."""
     pkg = os.path.join(ROOT, "bit_nf4_quantised_codebook_b200")
