@@ -323,13 +323,27 @@ cudaError_t launch_merge_requantize(const qlora_nf4_weight &w, const uint16_t *A
   cudaError_t e = cudaFuncSetAttribute(k_merge_quant, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        static_cast<int>(smem));
   if (e != cudaSuccess) return e;
-  int per_sm = 0;
-  e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, k_merge_quant, 128, smem);
+  // Several CTAs per SM need the largest shared-memory share of the on-chip memory;
+  // without this hint the driver may configure room for only one.
+  e = cudaFuncSetAttribute(k_merge_quant, cudaFuncAttributePreferredSharedMemoryCarveout,
+                           cudaSharedmemCarveoutMaxShared);
   if (e != cudaSuccess) return e;
-  int dev = 0, sms = 148;
-  if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  // CTAs resident per SM, from registers, shared memory and TMEM columns.
+  cudaFuncAttributes fa;
+  if ((e = cudaFuncGetAttributes(&fa, k_merge_quant)) != cudaSuccess) return e;
+  int dev = 0, sms = 148, smem_sm = 0, reserved = 0;
+  if ((e = cudaGetDevice(&dev)) != cudaSuccess) return e;
+  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  cudaDeviceGetAttribute(&smem_sm, cudaDevAttrMaxSharedMemoryPerMultiprocessor, dev);
+  cudaDeviceGetAttribute(&reserved, cudaDevAttrReservedSharedMemoryPerBlock, dev);
+  const int regs_warp = (fa.numRegs * 32 + 255) / 256 * 256;
+  const int by_regs = regs_warp > 0 ? 65536 / (regs_warp * 4) : 1;
+  const int by_smem = static_cast<int>(smem_sm / (smem + fa.sharedSizeBytes + reserved));
+  int per_sm = by_regs < by_smem ? by_regs : by_smem;
+  if (per_sm > 512 / kCols) per_sm = 512 / kCols;
+  if (per_sm < 1) per_sm = 1;
   const int64_t tiles = ((w.N + kRows - 1) / kRows) * (w.K / kCols);
-  const int64_t slots = static_cast<int64_t>(per_sm > 0 ? per_sm : 1) * sms;
+  const int64_t slots = static_cast<int64_t>(per_sm) * sms;
   const int64_t grid = tiles < slots ? tiles : slots;
   const TimingHooks &hk = timing_hooks();
   if (hk.fwd_begin) cudaEventRecord(hk.fwd_begin, st);
