@@ -584,6 +584,10 @@ def run_adamw(args):
 
 
 MERGE_SHAPES = ADAMW_SHAPES  # the seven linears of one LLaMA-7B decoder layer
+# ncu DRAM read + write of the merge-and-code kernel over one step's seven launches
+# (profiles/merge_requantize_llama7b_layer.md), valid for the sources it was taken from.
+MERGE_SOURCES = ["merge.cu", "nf4_decode.cuh", "nf4_quant.cuh", "ptx.cuh", "launch.cuh"]
+MERGE_TRAFFIC = {"sources_sha1": "4e714f616c7e4e56f4c0d477b522210425681dd2", "bytes_per_step": 117_096_000}
 
 
 def merge_bytes(N: int, K: int, r: int) -> int:
@@ -730,9 +734,12 @@ def run_merge(args):
                    "l2": f"{ncopy} copies of the layer in rotation; each step reads and writes "
                          f"{step_bytes / 1e6:.0f} MB (> L2)"},
         "kernels": {"merge_kernel_ms_per_step": round(kern_ms, 5)},
-        "roofline": {"kernel": "k_merge_quant", "bound": "hbm", "achieved": round(achieved, 1), "peak": hbm,
-                     "unit": "GB/s", "frac": round(achieved / hbm, 4), "peak_source": f"{peak_src} HBM copy",
-                     "traffic": None, "traffic_unit": "bytes per launch (ncu dram read+write)"},
+        "roofline": {"kernel": "k_merge_quant (7 launches per step)", "bound": "hbm", "achieved": round(achieved, 1),
+                     "peak": hbm, "unit": "GB/s", "frac": round(achieved / hbm, 4),
+                     "peak_source": f"{peak_src} HBM copy",
+                     "traffic": (MERGE_TRAFFIC["bytes_per_step"] if MERGE_TRAFFIC["sources_sha1"] ==
+                                 kernel_sources_sha1(MERGE_SOURCES) else None),
+                     "traffic_unit": "bytes per step, 7 launches (ncu dram read+write)"},
         "e2e": {"value": round(step_bytes / (e2e_ms * 1e-3) / 1e9, 2), "unit": "GB/s",
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": e2e_steps},
         "gpu_launches": int(launches),
