@@ -1,0 +1,48 @@
+"""The byte counts bench.py divides by, checked against the sizes the library
+itself reports for the stored formats (host calls, no GPU) and against the
+oracle's storage accounting."""
+import ctypes
+import itertools
+
+import pytest
+
+import bench
+from oracle import formats as F
+from oracle import nf4
+
+
+@pytest.fixture(scope="module")
+def api():
+    from bit_nf4_quantised_codebook_b200 import build
+    build.build()
+    from bit_nf4_quantised_codebook_b200 import api as a
+    return a
+
+
+def test_format_stored_bytes_match_library_sizes(api):
+    L = api.lib()
+    for (cb, block, dq), (n, k) in itertools.product(
+            itertools.product(bench.FORMAT_CODEBOOKS, bench.FORMAT_BLOCKS, bench.FORMAT_DQ),
+            [(4096, 4096), (40, 1536), (11008, 4096)]):
+        f = api._Format(api.CODEBOOKS[cb], block, api.DQ_MODES[dq])
+        a, b, c = ctypes.c_size_t(), ctypes.c_size_t(), ctypes.c_size_t()
+        assert L.qlora_format_sizes(ctypes.byref(f), n, k, ctypes.byref(a), ctypes.byref(b), ctypes.byref(c)) == 0
+        mean = 0 if dq == "none" else 4
+        assert bench.format_stored_bytes(n, k, block, dq) == a.value + b.value + c.value + mean
+        bits = F.storage_bits_per_weight(block, dq, n, k)
+        assert abs(8 * bench.format_stored_bytes(n, k, block, dq) / (n * k) - bits) < 1e-12
+
+
+def test_merge_bytes(api):
+    for _, n, k in bench.MERGE_SHAPES:
+        cb, qb, sb = api.qlora_nf4_sizes(n, k)
+        packed = cb + qb + sb + 4
+        assert packed == nf4.storage_bytes(n, k)
+        assert bench.merge_bytes(n, k, 64) == 2 * packed + 2 * 64 * (k + n)
+        nb = n * k // 64
+        assert bench.merge_kernel_bytes(n, k, 64) == packed + 2 * 64 * (k + n) + n * k // 2 + 4 * nb
+
+
+def test_adamw_bytes_per_parameter():
+    # read p, g, m, v (float32); write p, m, v (float32) and the bfloat16 copy
+    assert bench.ADAMW_BYTES_PER_PARAM == 4 * 4 + 3 * 4 + 2
