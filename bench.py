@@ -271,6 +271,20 @@ def run_ours(args):
     ms_step = ms / args.steps
     value = whole_job_rate(flops, world, ms_step * 1e-3) / 1e12
 
+    # the quantiser alone (block kernel, mean, E4M3 constants), events around each call
+    # and a write of a buffer larger than L2 before it, so that W comes from HBM
+    qsteps = max(3, min(50, args.steps))
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    qev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(qsteps)]
+    for i in range(qsteps):
+        flush.zero_()
+        qev[i][0].record()
+        api.qlora_quantize(sets[i % NSETS]["W"], out=wq, ws=ws_q, dev_err=err)
+        qev[i][1].record()
+    torch.cuda.synchronize()
+    q_ms = sum(a.elapsed_time(b) for a, b in qev) / qsteps
+    del flush
+
     # end to end through the public API with pinned host buffers: H2D of the step's
     # inputs (W, X, A, B, dY), the step, D2H of its results (Y, dX, dA, dB)
     e2e_steps = max(3, min(20, args.steps // 10))
@@ -323,7 +337,12 @@ def run_ours(args):
                    "step": "quantise(W) + forward + backward",
                    "l2": f"inputs larger than L2: {NSETS} rotating input sets (W, X, dY 33.5 MB each) + 67 MB outputs"},
         "packed_weight_gbs": round(2 * packed / (ms_step * 1e-3) / 1e9, 2),
-        "kernels": {"fwd_fused_ms": round(fwd_ms, 4), "bwd_fused_ms": round(bwd_ms, 4)},
+        "kernels": {"fwd_fused_ms": round(fwd_ms, 4), "bwd_fused_ms": round(bwd_ms, 4),
+                    "quantize_ms": round(q_ms, 4)},
+        "quantiser": {"params_per_s": round(N * K / (q_ms * 1e-3), 1),
+                      "gbs": round((2 * N * K + packed) / (q_ms * 1e-3) / 1e9, 1),
+                      "hbm_frac": round((2 * N * K + packed) / (q_ms * 1e-3) / 1e9 / hbm, 4),
+                      "bytes": "bf16 W read + stored weight written, per call (3 kernels), L2 flushed before each"},
         "roofline": {"kernel": f"fused dequant GEMM ({dom})", "bound": "tensor",
                      "achieved": round(achieved, 2), "peak": bf16_burst, "unit": "TFLOP/s",
                      "frac": round(achieved / bf16_burst, 4), "peak_source": f"{peak_src} bf16 burst",
