@@ -14,7 +14,7 @@ Sources (web pages on QLoRA):
        (tildalice.io) §What Would Trip You Up in Practice: smaller blocks give
        better precision and more overhead, larger blocks the reverse.
 
-Readings (also listed in the design doc):
+Readings taken where the pages are silent:
   * Int4: the symmetric absmax integer grid, levels k/7 for k = -7..7 (the
     int8 recipe of §Quantize in blocks with 7 in place of 127; the level
     -8/7 completes the 16-entry table and is never the nearest to a value in

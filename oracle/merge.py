@@ -11,7 +11,7 @@ Sources (web pages on QLoRA):
        X·W_hatᵀ + s·(X·A)·B, so the weight the adapter adds is s·(A·B)ᵀ
        (this library stores W as [N, K], A as [K, r], B as [r, N]).
 
-Readings (also listed in the design doc):
+Readings taken where the pages are silent:
   * merged weight: W_eff[n, k] = W_hat[n, k] + s·sum_j A[k, j]·B[j, n], the
     exact value rounded once to float32 (round to nearest even), then stored
     as bfloat16 (round to nearest even) — bfloat16 being the type the

@@ -10,8 +10,7 @@ Sources (web pages on QLoRA):
        (tildalice.io) §What QLoRA Actually Does.
   [P5] "4-bit QLoRA" glossary (inferensys.com), double quantization entry.
 
-Readings taken where the pages are silent or garbled (each also listed in
-DESIGN.md):
+Readings taken where the pages are silent or garbled:
   * code points: the offset recipe of [P2] §NormalFloat (the literal
     ``Q^-1(i/2^k)`` of [P1] is infinite at i = 0); computed in float64,
     normalised by the largest magnitude, then rounded to float32;
