@@ -1040,7 +1040,8 @@ def run_reference(args):
     world, rank, _ = _dist()
     if rank != 0:
         return
-    budget = 120.0 / max(1, args.steps + args.warmup)
+    # host seconds for the whole run (about two minutes; a test shortens it)
+    budget = float(os.environ.get("QLORA_REFERENCE_SECONDS", "120")) / max(1, args.steps + args.warmup)
     n = 16
     dt, _ = _oracle_sample(n, n)
     while n < 1024 and dt * 2.2 < budget:
