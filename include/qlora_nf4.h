@@ -12,6 +12,10 @@
  *   - §The QLoRA layer, end to end: Y = X·W + s·(X·L1)·L2 with W dequantised
  *     to bfloat16 on the fly; backward gives dX through W and the adapter,
  *     and gradients for L1, L2 only.
+ * Around the layer: the optimiser step of the adapters (qlora_adamw_step),
+ * merging a trained adapter into the quantised base and requantising
+ * (qlora_merge_requantize), and the storage-format variants the pages compare
+ * NF4 with (qlora_quantize_format and its companions).
  *
  * Conventions of this library:
  *   W  [N, K]  frozen weight, bfloat16, row-major (out x in, as a framework
@@ -38,7 +42,8 @@
  *                   w_hat = bf16_rn(float32(level[code] · c2_hat_b)).
  *
  * bfloat16 tensors are passed as uint16_t bit patterns.  All sizes are in
- * elements unless stated.  Every device pointer must be 16-byte aligned.
+ * elements unless stated.  Every device pointer must be 16-byte aligned unless
+ * its entry point says otherwise.
  * `stream` is a cudaStream_t (NULL = legacy default stream).  Every call is
  * asynchronous on `stream`, never synchronises and never allocates.
  *
@@ -69,7 +74,7 @@ typedef enum {
 } qlora_status;
 
 /* Bits OR-ed into *dev_err by kernels. */
-#define QLORA_DEVERR_NONFINITE 1   /* the weight given to qlora_quantize held Inf/NaN */
+#define QLORA_DEVERR_NONFINITE 1   /* a weight to quantise (given, or merged) held Inf/NaN */
 #define QLORA_DEVERR_TIMEOUT   2   /* a pipeline wait exceeded its bound; outputs are undefined */
 
 typedef struct qlora_nf4_weight {
