@@ -115,6 +115,8 @@ class ClockSampler:
             time.sleep(0.3)
         except Exception:
             self.proc = None
+            if self.path and os.path.exists(self.path):
+                os.unlink(self.path)
 
     def stop(self) -> dict:
         if self.proc is None:

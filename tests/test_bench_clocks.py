@@ -46,3 +46,4 @@ def test_clock_sampler_without_nvidia_smi(tmp_path, monkeypatch):
     s.mark_end()
     out = s.stop()
     assert out["reasons"] == ["unavailable"] and out["sm_mhz"] is None
+    assert not os.path.exists(s.path)  # no sample file left behind
