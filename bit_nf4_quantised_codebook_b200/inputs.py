@@ -27,8 +27,11 @@ import torch
 
 
 def to_bf16_bits(x: np.ndarray) -> np.ndarray:
-    """Round a float array to bfloat16 (RNE, torch's conversion); return uint16 bits."""
-    t = torch.from_numpy(np.ascontiguousarray(x, dtype=np.float32))
+    """Round a float array to float32 and then to bfloat16 (both round to
+    nearest-even, torch's conversions, run on all host threads); return uint16 bits."""
+    t = torch.from_numpy(np.ascontiguousarray(x))
+    if t.dtype != torch.float32:
+        t = t.to(torch.float32)
     return t.to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16).copy()
 
 

@@ -47,6 +47,16 @@ def backward(x_bits, dy_bits, w_hat_bits, a_bits, b_bits, s: float) -> dict:
     return {"dX": dX, "dA": dA, "dB": dB, "U": U, "T": T}
 
 
+def adapter_grads(x_bits, dy_bits, a_bits, b_bits, s: float) -> dict:
+    """dA = s·Xᵀ·(dY·Bᵀ) and dB = s·(X·A)ᵀ·dY without dX: the adapter gradients
+    need no W_hat, so they stay cheap at shapes where dY·W_hat is not."""
+    X = bf16_to_f64(x_bits)
+    dY = bf16_to_f64(dy_bits)
+    A = bf16_to_f64(a_bits)
+    B = bf16_to_f64(b_bits)
+    return {"dA": s * (X.T @ (dY @ B.T)), "dB": s * ((X @ A).T @ dY)}
+
+
 def backward_dx_rows(rows, dy_bits, w_hat_bits, a_bits, b_bits, s: float) -> np.ndarray:
     """dX restricted to the given token rows (dX rows depend only on dY rows)."""
     dY = bf16_to_f64(dy_bits)[rows]

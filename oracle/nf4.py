@@ -268,12 +268,17 @@ def _round_fraction_to_f32(v: Fraction) -> np.float32:
     return r
 
 
-def reconstruct_c2(e: np.ndarray, s: np.ndarray, mu: np.float32) -> np.ndarray:
+def reconstruct_c2(e: np.ndarray, s: np.ndarray, mu: np.float32, groups: np.ndarray | None = None) -> np.ndarray:
     """Inner dequant of [P2] §The QLoRA layer: c2_hat_b = e_b * S_g + mu,
-    rounded once to float32 (the exact value, as a fused multiply-add gives)."""
+    rounded once to float32 (the exact value, as a fused multiply-add gives).
+    ``groups`` gives each entry of ``e`` its group (default: entry b is block b,
+    in group b // 256)."""
     e64 = e4m3_decode(e)
     nb = e64.size
-    sg = np.repeat(np.asarray(s, _F32).astype(_F64), GROUP)[:nb]
+    if groups is None:
+        sg = np.repeat(np.asarray(s, _F32).astype(_F64), GROUP)[:nb]
+    else:
+        sg = np.asarray(s, _F32).astype(_F64)[np.asarray(groups, np.int64)]
     p = e64 * sg                                # exact: <= 4 x 24 significant bits
     m = _F64(mu)
     tot = p + m
@@ -314,6 +319,46 @@ def quantize_nf4(w_bits: np.ndarray, levels: np.ndarray | None = None) -> dict:
 
 def dequantize_nf4(q: dict) -> np.ndarray:
     return dequantize(q["codes"], q["c2q"], q["c1"], q["mean"], q["levels"], q["N"], q["K"])
+
+
+def quantize_nf4_blocks(w_bits: np.ndarray, blocks, levels: np.ndarray | None = None) -> dict:
+    """quantize_nf4 evaluated only for the flat blocks listed in ``blocks``, for
+    tensors too large to quantise whole on the host in a test.  The steps are
+    those of quantize_nf4: the absmax of every block (the mean and the group
+    scales depend on all of them), the fixed-order mean, each group's scale
+    S_g = amax_g|c2 - mu| / 448; then, for the listed blocks only, the codes
+    (nearest level of w / c2) and the E4M3 constant of (c2 - mu) / S_g.
+    Returns the listed blocks' packed codes [len, 32], E4M3 constants and
+    absmax, every group scale, and the mean."""
+    n, k = w_bits.shape
+    if (n * k) % BLOCK:
+        raise ValueError("N*K must be a multiple of 64")
+    lv = nf4_levels() if levels is None else levels
+    blocks = np.asarray(blocks, np.int64).reshape(-1)
+    c2 = block_absmax(w_bits)
+    mu = fixed_order_mean(c2)
+    dev = (c2 - mu).astype(_F32)
+    nb = c2.size
+    ng = -(-nb // GROUP)
+    amax = np.zeros(ng * GROUP, _F32)
+    amax[:nb] = np.abs(dev)
+    s = (amax.reshape(ng, GROUP).max(axis=1) / _F32(E4M3_MAX)).astype(_F32)
+    sg = s[blocks // GROUP]
+    safe = np.where(sg == 0, _F32(1), sg).astype(_F32)
+    e = np.where(sg == 0, np.uint8(0), e4m3_encode((dev[blocks] / safe).astype(_F32))).astype(np.uint8)
+    codes, c2_sel = quantize_codes(np.asarray(w_bits).reshape(-1, BLOCK)[blocks], lv)
+    return {"N": n, "K": k, "blocks": blocks, "codes": pack_nibbles(codes).reshape(-1, BLOCK // 2),
+            "c2q": e, "c1": s, "mean": mu, "absmax": c2_sel, "levels": lv}
+
+
+def dequantize_nf4_blocks(qb: dict) -> np.ndarray:
+    """doubleDequant of the blocks held by a quantize_nf4_blocks result:
+    bfloat16 bits [len(blocks), 64]."""
+    codes = unpack_nibbles(qb["codes"]).reshape(-1, BLOCK)
+    c2h = reconstruct_c2(qb["c2q"], qb["c1"], qb["mean"], groups=qb["blocks"] // GROUP).astype(_F64)
+    q = np.asarray(qb["levels"], _F32).astype(_F64)
+    prod = (q[codes] * c2h[:, None]).astype(_F32)
+    return f32_to_bf16_rne(prod).reshape(-1, BLOCK)
 
 
 def storage_bytes(n: int, k: int, double_quant: bool = True) -> int:

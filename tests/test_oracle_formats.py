@@ -135,3 +135,22 @@ def test_int8_reconstruction_is_one_rounding():
         up = Fraction(float(np.nextafter(ch[b], np.float32(np.inf))))
         dn = Fraction(float(np.nextafter(ch[b], np.float32(-np.inf))))
         assert abs(got - exact) <= abs(up - exact) and abs(got - exact) <= abs(dn - exact)
+
+
+def test_error_stats_hand_computed():
+    """Values worked out by hand: a dropped square root, a missing division by
+    the weight's norm or a maximum taken along one axis only fails one of them."""
+    w = to_bf16_bits(np.array([[3.0, 4.0, 0.0, 0.0], [0.0, 0.0, 0.0, 0.0]]))
+    zero = to_bf16_bits(np.zeros((2, 4)))
+    # W_hat = 0: the error is W itself, |W| = 5
+    assert F.error_stats(w, zero) == {"rel_fro": 1.0, "max_abs": 4.0, "mean_abs": 7.0 / 8.0}
+    # W_hat = W / 2 (exact in bfloat16): error W / 2
+    half = to_bf16_bits(np.array([[1.5, 2.0, 0.0, 0.0], [0.0, 0.0, 0.0, 0.0]]))
+    assert F.error_stats(w, half) == {"rel_fro": 0.5, "max_abs": 2.0, "mean_abs": 7.0 / 16.0}
+    # error [[0.5, 0], [0, -4]] on W = [[1, 0], [0, -6]]: |d|^2 = 16.25, |W|^2 = 37;
+    # the largest error is in the second row and the second column
+    w2 = to_bf16_bits(np.array([[1.0, 0.0], [0.0, -6.0]]))
+    h2 = to_bf16_bits(np.array([[0.5, 0.0], [0.0, -2.0]]))
+    st = F.error_stats(w2, h2)
+    assert abs(st["rel_fro"] - (65.0 / 148.0) ** 0.5) < 1e-15
+    assert st["max_abs"] == 4.0 and st["mean_abs"] == 4.5 / 4.0

@@ -33,9 +33,12 @@ def test_gradients_by_finite_differences(which):
     s = 2.0
     X, wh, A, B, dY = _case()
     g = linear.backward(X, dY, wh, A, B, s)
+    ga = linear.adapter_grads(X, dY, A, B, s)
     Xf, Wf, Af, Bf, dYf = (nf4.bf16_to_f64(t) for t in (X, wh, A, B, dY))
     base = {"X": Xf, "A": Af, "B": Bf}
     grad = {"X": g["dX"], "A": g["dA"], "B": g["dB"]}[which]
+    # the adapter-only form (no dX) is held to the same finite differences
+    grad2 = {"X": g["dX"], "A": ga["dA"], "B": ga["dB"]}[which]
     rng = np.random.default_rng(9)
     h = 0.5
     for _ in range(25):
@@ -47,6 +50,7 @@ def test_gradients_by_finite_differences(which):
         lm = _loss(args["X"], Wf, args["A"], args["B"], dYf, s)
         fd = (lp - lm) / (2 * h)
         assert abs(fd - grad[idx]) <= 1e-9 * (1 + abs(fd)), (which, idx, fd, grad[idx])
+        assert abs(fd - grad2[idx]) <= 1e-9 * (1 + abs(fd)), (which, idx, fd, grad2[idx])
 
 
 def test_forward_matches_definition_and_lora_term():

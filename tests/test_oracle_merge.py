@@ -149,3 +149,26 @@ def test_requantisation_error_bound():
     assert 0.0 < err["rel_fro"] < 0.2
     # the merge moved the weights: codes changed in some blocks
     assert not np.array_equal(q2["codes"], q["codes"])
+
+
+def test_requant_error_hand_computed():
+    """Two blocks whose round trip is worked out by hand.  Both blocks have
+    absmax 1, so the mean of the constants is 1, every deviation is 0, the
+    group scale is 0 and the reconstructed constant is exactly 1.  Row 0,
+    [1, 0, ...], is exact.  In row 1, [0.5, -1, 0, ...], -1 is level 0
+    exactly and 0.5 goes to the nearest level 0.4407098 (the next one up is
+    0.5626170), stored as bfloat16 0.44140625: error 0.05859375 at (1, 0).
+    |W| = sqrt(1 + 0.25 + 1) = 1.5."""
+    row0 = np.zeros(64)
+    row0[0] = 1.0
+    row1 = np.zeros(64)
+    row1[0], row1[1] = 0.5, -1.0
+    w = _bits(np.stack([row0, row1]))
+    q = nf4.quantize_nf4(w)
+    err = merge.requant_error(w, q)
+    assert err["max_abs"] == 0.05859375
+    assert abs(err["rel_fro"] - 0.05859375 / 1.5) < 1e-15
+    # weights already on the bfloat16 images of the levels (block absmax 1) round-trip exactly
+    lv = nf4.bf16_to_f64(_bits(nf4.nf4_levels().astype(np.float64)))
+    exact = _bits(np.tile(lv, 4).reshape(1, 64))
+    assert merge.requant_error(exact, nf4.quantize_nf4(exact)) == {"rel_fro": 0.0, "max_abs": 0.0}

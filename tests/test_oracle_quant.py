@@ -258,3 +258,22 @@ def test_quantize_output_sizes():
     assert q2["c1"].size == 2
     d = nf4.dequantize_nf4(q2)
     assert d.shape == (3, 6400)
+
+
+@pytest.mark.parametrize("n,k,frac,seed", [(40, 1536, 0.002, 31), (3, 11008, 0.001, 32), (1, 64, 0.0, 33)])
+def test_block_subset_equals_whole_tensor(n, k, frac, seed):
+    """The block-subset form gives, block for block, what the whole-tensor
+    quantiser and dequantiser give (rows straddling groups, a partial last
+    group, outliers, a single block)."""
+    w = weight_bf16(n, k, 0.02, seed, frac)
+    full = nf4.quantize_nf4(w)
+    wh = nf4.dequantize_nf4(full).reshape(-1, 64)
+    nb = n * k // 64
+    rng = np.random.default_rng(seed)
+    blocks = np.unique(np.concatenate([[0, nb - 1], rng.integers(0, nb, size=min(nb, 50))]))
+    sub = nf4.quantize_nf4_blocks(w, blocks)
+    assert np.array_equal(sub["codes"], full["codes"].reshape(-1, 32)[blocks])
+    assert np.array_equal(sub["c2q"], full["c2q"][blocks])
+    assert np.array_equal(sub["absmax"], full["absmax"][blocks])
+    assert np.array_equal(sub["c1"], full["c1"]) and sub["mean"] == full["mean"]
+    assert np.array_equal(nf4.dequantize_nf4_blocks(sub), wh[blocks])
