@@ -1,31 +1,36 @@
 """Benchmark of the QLoRA frozen-NF4 linear layer on B200.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
-                    [--workload proj7b | smallm --n N --m M | adamw]
+                    [--workload shapes_65b | llama7b_layer | proj7b | smallm --n N --m M
+                                | adamw | merge | formats] [--no-sub] [--no-cpu-baseline]
 
-One step = the whole hot path on one batch: NF4 + double quantisation of the
-bf16 weight, the forward (T = X·A, fused dequant GEMM Y = X·W_hatᵀ + sT·B) and
-the backward (U = dY·Bᵀ, fused dequant GEMM dX = dY·W_hat + sU·Aᵀ, dA, dB).
-Workload: a single 7B-class projection, W 4096 x 4096, X 4096 tokens
-(batch 4 x seq 1024), LoRA r = 64, alpha = 16, synthetic seeded inputs.
+Default workload: the 65B-class shapes.  The seven linears of one decoder
+layer with hidden size 8192 and FFN 22016 (q, k, v, o 8192 x 8192; gate, up
+22016 x 8192; down 8192 x 22016), weights N(0, 0.015) with 0.1% Student-t(3)
+outliers, quantised to NF4 + double quantisation once at load (the weights
+stay resident); 8192 tokens (batch 4 x seq 2048); LoRA r = 64, alpha = 16.
+One step = the forward of the seven linears (T = X·A, fused dequant GEMM
+Y = X·W_hatᵀ + sT·B) followed by their backward in reverse order (U = dY·Bᵀ,
+fused dequant GEMM dX = dY·W_hat + sU·Aᵀ, dA, dB).
 value = algorithmic fwd+bwd flops per step / device time (TFLOP/s).
 
---workload smallm: the decode-sized forward (K = 8192, N = 8192 or 28672 W rows,
-M = 1..64 tokens, r = 64; the weight quantised once and resident, rotated over
-enough copies to exceed L2); value = packed-weight bytes streamed per forward /
-device time (GB/s).
+The default line also carries sub-records, each measured the same way: the
+single 7B-class projection (4096^3, r = 64), the LLaMA-7B decoder layer's
+seven linears at 4096 tokens, the decode-sized forward (packed-weight GB/s
+and the fraction of HBM bandwidth of the small-M kernel) on 8192 x 8192 and
+28672 x 8192 at 1 and 16 tokens, and the quantiser (load-time cost) on the
+22016 x 8192 weight.
 
---workload adamw: the fused AdamW step on the 14 adapter tensors (r = 64) of
-one LLaMA-7B decoder layer (q, k, v, o: 4096 x 4096; gate, up: 11008 x 4096;
-down: 4096 x 11008), 5.0 M parameters, float32 master values and moments plus
-the bfloat16 copies, in one launch; value = bytes moved per step / device time
-(GB/s), 30 bytes per parameter.
+--workload smallm: the decode-sized forward alone (K = 8192, N = 8192 or 28672
+W rows, M = 1..64 tokens, r = 64).  --workload adamw / merge / formats: the
+optimiser step on the adapters, the adapter merge with requantisation and the
+storage-format study (see their functions).
 
-Multi-GPU: data parallel.  Every rank runs the layer on its own 4096-token
-shard (same weight, same adapters); the adapter gradients dA and dB, one
-float32 bucket, are summed over the ranks by one NCCL all-reduce per step, as
-a data-parallel training step needs.  value sums the ranks' work over the
-slowest rank's time (weak scaling).  Rank 0 prints one JSON line.
+Multi-GPU: data parallel over tokens.  Every rank runs the step on its own
+8192-token shard (its own seeds for X and dY; the same weights and adapters);
+the adapter gradients of all seven linears, one float32 bucket, are summed
+over the ranks by one NCCL all-reduce per step.  value sums the ranks' work
+over the slowest rank's time (weak scaling).  Rank 0 prints one JSON line.
 """
 from __future__ import annotations
 
@@ -45,7 +50,15 @@ if ROOT not in sys.path:
     sys.path.insert(0, ROOT)
 
 METRIC = "QLoRA linear fwd+bwd TFLOP/s; packed-weight GB/s; fraction of roofline"
-WORKLOAD = "single 7B-class projection: W 4096x4096 NF4+DQ, X 4096 tokens (4x1024), LoRA r=64 alpha=16"
+WORKLOADS = {
+    "shapes_65b": "65B-class shapes: q/k/v/o 8192x8192, gate/up 22016x8192, down 8192x22016, NF4+DQ, "
+                  "8192 tokens (4x2048), LoRA r=64 alpha=16, fwd+bwd of all 7",
+    "llama7b_layer": "LLaMA-7B decoder layer linears: q/k/v/o 4096x4096, gate/up 11008x4096, down 4096x11008, "
+                     "NF4+DQ, 4096 tokens (2x2048), LoRA r=64 alpha=16, fwd+bwd of all 7",
+    "proj7b": "single 7B-class projection: W 4096x4096 NF4+DQ, X 4096 tokens (4x1024), LoRA r=64 alpha=16, "
+              "fwd+bwd",
+}
+BATCH = {"shapes_65b": (4, 2048), "llama7b_layer": (2, 2048), "proj7b": (4, 1024)}
 
 
 def _peaks():
@@ -58,20 +71,20 @@ def _peaks():
         return 6650.0, 1590.0, 1400.0, "fallback"
 
 
-# DRAM traffic (read + write bytes per launch) of the fused dequant GEMMs from the
-# ncu capture summarised in profiles/fused_dequant_gemm_proj7b.md.  Reported only
-# while the kernel sources hash to the build that capture was taken of.
+# DRAM traffic (ncu dram__bytes_read.sum + dram__bytes_write.sum) of the dominant
+# kernels, from one-pass ncu launch-list captures, reported only while the kernel
+# sources hash to the build each capture was taken of (otherwise null).
+# Fused dequant GEMMs: `ncu --metrics gpu__time_duration.sum,dram__bytes_read.sum,
+# dram__bytes_write.sum --clock-control none -k regex:gemm_pair` over one step of
+# each layer set; bytes per step summed over the seven forward (fwd) or backward
+# (bwd) launches.
 KERNEL_SOURCES = ["gemm_pair.cuh", "gemm.cuh", "nf4_decode.cuh", "ptx.cuh", "launch.cuh", "linear.cu"]
-TRAFFIC_CAPTURE = {"sources_sha1": "118f0767b267fedf5a145b9c8a726560220b6710",
-                   "fwd_y": 46_729_344, "bwd_dx": 45_281_792}
-
-
-# Same for the small-M kernel (profiles/smallm_dequant_gemm_8192x8192_m16.md), per (N, M).
+TRAFFIC_CAPTURE = {"sources_sha1": None}
+# The small-M kernel: the same one-pass capture of `--workload smallm`, bytes per launch, per (N, M).
 SMALLM_SOURCES = ["gemm_smallm.cuh", "gemm.cuh", "nf4_decode.cuh", "ptx.cuh", "launch.cuh", "linear.cu"]
-SMALLM_TRAFFIC = {"sources_sha1": "be7e178431def2548439e796db2b1528aaaa2b5c", (8192, 16): 35_976_960}
-
-
-# Same for the AdamW kernel (profiles/adamw_llama7b_layer_adapters.md).
+SMALLM_TRAFFIC = {"sources_sha1": None}
+# The AdamW kernel: the same capture of `--workload adamw`, bytes per launch (the 150 MB working
+# set is only a little larger than L2, so part of the writes stay in L2).
 ADAMW_SOURCES = ["adamw.cu", "ptx.cuh", "launch.cuh"]
 ADAMW_TRAFFIC = {"sources_sha1": "0064428f763192ff27c64743df1b67afd4a73e71", "bytes": 90_732_000}
 
@@ -82,6 +95,12 @@ def kernel_sources_sha1(files=None) -> str:
         with open(os.path.join(ROOT, "bit_nf4_quantised_codebook_b200", "csrc", f), "rb") as fh:
             h.update(fh.read())
     return h.hexdigest()
+
+
+def _traffic(table, files, key):
+    if table.get("sources_sha1") and table["sources_sha1"] == kernel_sources_sha1(files):
+        return table.get(key)
+    return None
 
 
 class ClockSampler:
@@ -152,11 +171,32 @@ class ClockSampler:
                 "power_w_max": max((float(r[3]) for r in rows if r[3].replace(".", "").isdigit()), default=None)}
 
 
+def _gpu_sampler(local):
+    import torch
+    gpu_id = None
+    try:
+        gpu_id = "GPU-" + str(torch.cuda.get_device_properties(local).uuid)
+    except Exception:
+        pass
+    s = ClockSampler(gpu_id)
+    s.start()
+    return s
+
+
 def _dist():
     ws = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     local = int(os.environ.get("LOCAL_RANK", "0"))
     return ws, rank, local
+
+
+def _init_dist(world, local):
+    import torch
+    import torch.distributed as dist
+    from datetime import timedelta
+    torch.cuda.set_device(local)
+    if world > 1:
+        dist.init_process_group("nccl", timeout=timedelta(seconds=120), device_id=torch.device("cuda", local))
 
 
 def max_over_ranks(x: float, device) -> float:
@@ -169,214 +209,336 @@ def max_over_ranks(x: float, device) -> float:
 
 
 def whole_job_rate(work_per_replica: float, world: int, seconds: float) -> float:
-    """Replicas only: every rank runs the same workload, so the job does `world` times the work."""
+    """Every rank does the same amount of work (its own shard or replica), so the job does `world` times it."""
     return work_per_replica * world / seconds
 
 
-def run_ours(args):
+def grad_bucket(shapes, device):
+    """One float32 bucket holding the adapter gradients dA [K, r] and dB [r, N]
+    of every linear, so that a data-parallel step sums them with one
+    all-reduce.  shapes = [(K, r, N), ...]; returns (bucket, [(dA, dB), ...])."""
     import torch
+    total = sum(k * r + r * n for k, r, n in shapes)
+    bucket = torch.zeros(total, dtype=torch.float32, device=device)
+    views, off = [], 0
+    for k, r, n in shapes:
+        dA = bucket[off:off + k * r].view(k, r)
+        off += k * r
+        dB = bucket[off:off + r * n].view(r, n)
+        off += r * n
+        views.append((dA, dB))
+    return bucket, views
+
+
+def allreduce_grads(bucket) -> None:
+    """The exchange step of data parallelism: dA and dB are sums over tokens, so
+    the ranks' shard gradients add up to the whole batch's (one sum all-reduce)."""
     import torch.distributed as dist
-    from datetime import timedelta
+    dist.all_reduce(bucket)
 
-    from bit_nf4_quantised_codebook_b200 import api, inputs
 
-    world, rank, local = _dist()
-    torch.cuda.set_device(local)
-    if world > 1:
-        dist.init_process_group("nccl", timeout=timedelta(seconds=120), device_id=torch.device("cuda", local))
-    api.lib()
-    dev = torch.device("cuda", local)
-    case = inputs.proj_7b()
-    M, N, K, r, s = case.M, case.N, case.K, case.r, case.s
-    flops = case.flops_fwd() + case.flops_bwd()
+# ---------------------------------------------------------------- inputs
+def _gen_tensor(kind: str, fields: dict):
+    """One seeded input tensor (bfloat16 bits) of a linear; runs in a worker process."""
+    from bit_nf4_quantised_codebook_b200 import inputs
+    return getattr(inputs.LinearCase(**fields), kind)()
 
-    # Input sets rotated so that consecutive steps never find their inputs in L2
-    # (one set: W 33.5 MB + X 33.5 MB + dY 33.5 MB; outputs 67 MB more).
-    NSETS = 3
-    sets = []
-    for i in range(NSETS):
-        c = inputs.LinearCase(case.name, M, N, K, r, case.alpha, case.w_std, case.a_std, case.b_std,
-                              seed=case.seed + 10 * i)
-        sets.append({k: api.bits_to_tensor(getattr(c, k)(), dev) for k in ("W", "X", "A", "B", "dY")})
-    wq = api.alloc_weight(N, K, dev)
-    Y = torch.empty(M, N, dtype=torch.bfloat16, device=dev)
-    sT = torch.empty(M, r, dtype=torch.bfloat16, device=dev)
-    dX = torch.empty(M, K, dtype=torch.bfloat16, device=dev)
-    # dA and dB share one float32 bucket: with several ranks (data parallel, one token
-    # shard per rank) the adapter gradients are summed by one all-reduce per step
-    gbucket = torch.empty(K * r + r * N, dtype=torch.float32, device=dev)
-    dA = gbucket[:K * r].view(K, r)
-    dB = gbucket[K * r:].view(r, N)
-    ws_q = torch.empty(api.qlora_workspace_size(api.QLORA_OP_QUANTIZE, 0, N, K, 0), dtype=torch.uint8, device=dev)
-    ws_f = torch.empty(api.qlora_workspace_size(api.QLORA_OP_FORWARD, M, N, K, r), dtype=torch.uint8, device=dev)
-    ws_b = torch.empty(api.qlora_workspace_size(api.QLORA_OP_BACKWARD, M, N, K, r), dtype=torch.uint8, device=dev)
-    err = api.new_error_word(dev)
 
-    def step(i, Win=None, Xin=None, Ain=None, Bin=None, dYin=None):
-        st = sets[i % NSETS]
-        Wt = st["W"] if Win is None else Win
-        Xt = st["X"] if Xin is None else Xin
-        At = st["A"] if Ain is None else Ain
-        Bt = st["B"] if Bin is None else Bin
-        dYt = st["dY"] if dYin is None else dYin
-        api.qlora_quantize(Wt, out=wq, ws=ws_q, dev_err=err)
-        api.qlora_linear_forward(wq, Xt, At, Bt, s, Y=Y, T_save=sT, ws=ws_f, dev_err=err)
-        api.qlora_linear_backward(wq, Xt, dYt, At, Bt, s, T_saved=sT, dX=dX, dA=dA, dB=dB, ws=ws_b, dev_err=err)
+def _fields(c) -> dict:
+    return dict(name=c.name, M=c.M, N=c.N, K=c.K, r=c.r, alpha=c.alpha, w_std=c.w_std, a_std=c.a_std,
+                b_std=c.b_std, outlier_frac=c.outlier_frac, seed=c.seed)
+
+
+def tensor_key(kind: str, c) -> tuple:
+    """Inputs that the seeded recipe makes identical (same generator seed, shape
+    and distribution) share one key and are generated once."""
+    if kind == "W":
+        return ("W", c.N, c.K, c.w_std, c.outlier_frac, c.seed)
+    if kind == "X":
+        return ("X", c.M, c.K, c.seed)
+    if kind == "A":
+        return ("A", c.K, c.r, c.a_std, c.seed)
+    if kind == "B":
+        return ("B", c.r, c.N, c.b_std, c.seed)
+    return ("dY", c.M, c.N, c.seed)
+
+
+def generate(requests, workers: int) -> dict:
+    """requests = {key: (kind, case)} -> {key: bfloat16 bits}; independent tensors
+    are drawn in parallel worker processes (spawned, so safe beside CUDA)."""
+    specs = {k: (kind, _fields(c)) for k, (kind, c) in requests.items()}
+    if workers > 1 and len(specs) > 1:
+        import multiprocessing as mp
+        from concurrent.futures import ProcessPoolExecutor
+        with ProcessPoolExecutor(max_workers=min(workers, len(specs)), mp_context=mp.get_context("spawn")) as ex:
+            futs = {k: ex.submit(_gen_tensor, *v) for k, v in specs.items()}
+            return {k: f.result() for k, f in futs.items()}
+    return {k: _gen_tensor(*v) for k, v in specs.items()}
+
+
+def _workers(world: int) -> int:
+    return max(1, min(8, (os.cpu_count() or 1) // max(1, world)))
+
+
+def shard_case(c, rank: int):
+    """The case whose X and dY are rank `rank`'s token shard (other seeds); rank 0 keeps the configuration's."""
+    from bit_nf4_quantised_codebook_b200 import inputs
+    return c if rank == 0 else inputs.LinearCase(c.name, c.M, c.N, c.K, c.r, c.alpha, c.w_std, c.a_std, c.b_std,
+                                                 c.outlier_frac, c.seed + 1000 * rank)
+
+
+def fused_flops(c) -> tuple[float, float]:
+    """Algorithmic flops of the two fused dequant GEMM launches of one linear:
+    forward X·W_hatᵀ + sT·B and backward dY·W_hat + sU·Aᵀ."""
+    return (2.0 * c.M * c.N * c.K + 2.0 * c.M * c.r * c.N, 2.0 * c.M * c.N * c.K + 2.0 * c.M * c.r * c.K)
+
+
+# ---------------------------------------------------------------- layer sets (fwd + bwd)
+class LayerSet:
+    """The linears of one workload on the device: weights quantised once and
+    resident, every linear's own input, output and gradient buffers, and one
+    training step over them (forwards in order, backwards in reverse)."""
+
+    def __init__(self, cases, dev, rank: int = 0, world: int = 1):
+        import torch
+        from bit_nf4_quantised_codebook_b200 import api
+        self.api = api
+        self.cases = list(cases)
+        self.dev = dev
+        xcases = [shard_case(c, rank) for c in self.cases]
+        req = {}
+        for c, xc in zip(self.cases, xcases):
+            for kind in ("W", "A", "B"):
+                req[tensor_key(kind, c)] = (kind, c)
+            for kind in ("X", "dY"):
+                req[tensor_key(kind, xc)] = (kind, xc)
+        host = generate(req, _workers(world))
+        self.err = api.new_error_word(dev)
+        ws_q = torch.empty(max(api.qlora_workspace_size(api.QLORA_OP_QUANTIZE, 0, c.N, c.K, 0) for c in self.cases),
+                           dtype=torch.uint8, device=dev)
+        self.ws_f = torch.empty(max(16, max(api.qlora_workspace_size(api.QLORA_OP_FORWARD, c.M, c.N, c.K, c.r)
+                                            for c in self.cases)), dtype=torch.uint8, device=dev)
+        self.ws_b = torch.empty(max(16, max(api.qlora_workspace_size(api.QLORA_OP_BACKWARD, c.M, c.N, c.K, c.r)
+                                            for c in self.cases)), dtype=torch.uint8, device=dev)
+        self.bucket, views = grad_bucket([(c.K, c.r, c.N) for c in self.cases], dev)
+        self.lin = []
+        for c, xc, (dA, dB) in zip(self.cases, xcases, views):
+            W = api.bits_to_tensor(host[tensor_key("W", c)], dev)
+            q = api.qlora_quantize(W, ws=ws_q, dev_err=self.err)
+            del W
+            L = {"case": c, "q": q, "dA": dA, "dB": dB,
+                 "X": api.bits_to_tensor(host[tensor_key("X", xc)], dev),
+                 "dY": api.bits_to_tensor(host[tensor_key("dY", xc)], dev),
+                 "A": api.bits_to_tensor(host[tensor_key("A", c)], dev),
+                 "B": api.bits_to_tensor(host[tensor_key("B", c)], dev),
+                 "Y": torch.empty(c.M, c.N, dtype=torch.bfloat16, device=dev),
+                 "sT": torch.empty(c.M, c.r, dtype=torch.bfloat16, device=dev),
+                 "dX": torch.empty(c.M, c.K, dtype=torch.bfloat16, device=dev)}
+            self.lin.append(L)
+        del host, ws_q
+        torch.cuda.synchronize()
+        self.check("quantisation at load")
+
+    def check(self, what: str) -> None:
+        import torch
+        torch.cuda.synchronize()
+        if int(self.err[0].item()) != 0:
+            raise RuntimeError(f"device error word {int(self.err[0].item())} during {what}")
+
+    def flops(self) -> float:
+        return sum(c.flops_fwd() + c.flops_bwd() for c in self.cases)
+
+    def packed_bytes(self) -> int:
+        return sum(L["q"].nbytes() for L in self.lin)
+
+    def step(self, ev=None) -> None:
+        api = self.api
+        for j, L in enumerate(self.lin):
+            if ev is not None:
+                api.qlora_set_timing_events(*ev[j])
+            api.qlora_linear_forward(L["q"], L["X"], L["A"], L["B"], L["case"].s, Y=L["Y"], T_save=L["sT"],
+                                     ws=self.ws_f, dev_err=self.err)
+        for j in reversed(range(len(self.lin))):
+            L = self.lin[j]
+            if ev is not None:
+                api.qlora_set_timing_events(*ev[j])
+            api.qlora_linear_backward(L["q"], L["X"], L["dY"], L["A"], L["B"], L["case"].s, T_saved=L["sT"],
+                                      dX=L["dX"], dA=L["dA"], dB=L["dB"], ws=self.ws_b, dev_err=self.err)
+        if ev is not None:
+            api.qlora_set_timing_events()
+
+    def measure(self, steps: int, warmup: int, world: int, local: int, e2e_steps: int = 3) -> dict:
+        """Warm-up, K timed steps (barrier + synchronize on both sides, max over
+        ranks), a second loop with events around every fused dequant GEMM, and
+        the end-to-end loop through pinned host buffers."""
+        import torch
+        import torch.distributed as dist
+        api = self.api
+
+        def one(ev=None):
+            self.step(ev)
+            if world > 1:
+                allreduce_grads(self.bucket)
+
+        for _ in range(warmup):
+            one()
+        self.check("warm-up")
+        sampler = _gpu_sampler(local)
         if world > 1:
-            dist.all_reduce(gbucket)  # sum of the ranks' adapter gradients (NCCL)
+            dist.barrier()
+        torch.cuda.synchronize()
+        launches0 = api.qlora_kernel_launch_count()
+        sampler.mark_start()
+        t0 = torch.cuda.Event(enable_timing=True)
+        t1 = torch.cuda.Event(enable_timing=True)
+        t0.record()
+        for _ in range(steps):
+            one()
+        t1.record()
+        torch.cuda.synchronize()
+        sampler.mark_end()
+        launches = api.qlora_kernel_launch_count() - launches0
+        if world > 1:
+            dist.barrier()
+        clocks = sampler.stop()
+        ms = t0.elapsed_time(t1)
+        if world > 1:
+            ms = max_over_ranks(ms, self.dev)
+        self.check("timing")
 
-    for i in range(args.warmup):
-        step(i)
-    torch.cuda.synchronize()
-    if int(err[0].item()) != 0:
-        raise RuntimeError(f"device error word {int(err[0].item())} during warm-up")
+        # the fused dequant GEMMs alone: events the library records around each launch
+        # (a separate loop, since an event between two kernels ends their programmatic overlap)
+        ksteps = max(1, min(steps, 10))
+        nl = len(self.lin)
+        ev = [[[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(nl)] for _ in range(ksteps)]
+        for row in ev:  # torch creates a CUDA event at its first record; the library records them afterwards
+            for quad in row:
+                for e in quad:
+                    e.record()
+        for i in range(ksteps):
+            one(ev[i])
+        torch.cuda.synchronize()
+        fwd_ms = [sum(ev[i][j][0].elapsed_time(ev[i][j][1]) for i in range(ksteps)) / ksteps for j in range(nl)]
+        bwd_ms = [sum(ev[i][j][2].elapsed_time(ev[i][j][3]) for i in range(ksteps)) / ksteps for j in range(nl)]
 
-    # dominant-kernel events (fused dequant GEMMs), one pair per step
-    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
-    for quad in ev:          # torch creates events lazily: record once so each has a handle
-        for e in quad:
-            e.record()
-    gpu_id = None
-    try:
-        gpu_id = "GPU-" + str(torch.cuda.get_device_properties(local).uuid)
-    except Exception:
-        pass
-    sampler = ClockSampler(gpu_id)
-    sampler.start()
-    if world > 1:
-        dist.barrier()
-    torch.cuda.synchronize()
-    launches0 = api.qlora_kernel_launch_count()
-    sampler.mark_start()
-    t0 = torch.cuda.Event(enable_timing=True)
-    t1 = torch.cuda.Event(enable_timing=True)
-    t0.record()
-    for i in range(args.steps):
-        api.qlora_set_timing_events(*ev[i])
-        step(i)
-    t1.record()
-    torch.cuda.synchronize()
-    sampler.mark_end()
-    api.qlora_set_timing_events()
-    launches = api.qlora_kernel_launch_count() - launches0
-    if world > 1:
-        dist.barrier()
-    clocks = sampler.stop()
-    ms = t0.elapsed_time(t1)
-    fwd_ms = sum(e[0].elapsed_time(e[1]) for e in ev) / args.steps
-    bwd_ms = sum(e[2].elapsed_time(e[3]) for e in ev) / args.steps
-    if world > 1:
-        ms = max_over_ranks(ms, dev)
-    torch.cuda.synchronize()
-    if int(err[0].item()) != 0:
-        raise RuntimeError(f"device error word {int(err[0].item())} during timing")
-    ms_step = ms / args.steps
-    value = whole_job_rate(flops, world, ms_step * 1e-3) / 1e12
+        # end to end through the public API: every linear's X and dY in from pinned
+        # host memory, the step, Y, dX and the adapter gradients back out
+        h_in = [{k: torch.empty_like(L[k], device="cpu").pin_memory() for k in ("X", "dY")} for L in self.lin]
+        for h, L in zip(h_in, self.lin):
+            for k in h:
+                h[k].copy_(L[k])
+        h_out = [{k: torch.empty_like(L[k], device="cpu").pin_memory() for k in ("Y", "dX")} for L in self.lin]
+        h_grad = torch.empty_like(self.bucket, device="cpu").pin_memory()
+        h2d = sum(t.numel() * t.element_size() for h in h_in for t in h.values())
+        d2h = sum(t.numel() * t.element_size() for h in h_out for t in h.values()) + h_grad.numel() * 4
+        if world > 1:
+            dist.barrier()
+        torch.cuda.synchronize()
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        e0.record()
+        for _ in range(e2e_steps):
+            for h, L in zip(h_in, self.lin):
+                for k in h:
+                    L[k].copy_(h[k], non_blocking=True)
+            one()
+            for h, L in zip(h_out, self.lin):
+                for k in h:
+                    h[k].copy_(L[k], non_blocking=True)
+            h_grad.copy_(self.bucket, non_blocking=True)
+        e1.record()
+        torch.cuda.synchronize()
+        e2e_ms = e0.elapsed_time(e1)
+        if world > 1:
+            e2e_ms = max_over_ranks(e2e_ms, self.dev)
+        self.check("the end-to-end loop")
+        return {"ms_step": ms / steps, "fwd_ms": fwd_ms, "bwd_ms": bwd_ms, "launches": int(launches),
+                "clocks": clocks, "e2e_ms_step": e2e_ms / e2e_steps, "e2e_steps": e2e_steps, "h2d": h2d,
+                "d2h": d2h}
 
-    # the quantiser alone (block kernel, mean, E4M3 constants), events around each call
-    # and a write of a buffer larger than L2 before it, so that W comes from HBM
-    qsteps = max(3, min(50, args.steps))
-    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
-    qev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(qsteps)]
-    for i in range(qsteps):
-        flush.zero_()
-        qev[i][0].record()
-        api.qlora_quantize(sets[i % NSETS]["W"], out=wq, ws=ws_q, dev_err=err)
-        qev[i][1].record()
-    torch.cuda.synchronize()
-    q_ms = sum(a.elapsed_time(b) for a, b in qev) / qsteps
-    del flush
 
-    # end to end through the public API with pinned host buffers: H2D of the step's
-    # inputs (W, X, A, B, dY), the step, D2H of its results (Y, dX, dA, dB)
-    e2e_steps = max(3, min(20, args.steps // 10))
-    host_in = {k: torch.empty_like(v, device="cpu").pin_memory() for k, v in sets[0].items()}
-    for k in host_in:
-        host_in[k].copy_(sets[0][k])
-    dev_in = {k: torch.empty_like(v) for k, v in sets[0].items()}
-    host_out = [torch.empty_like(t, device="cpu").pin_memory() for t in (Y, dX, dA, dB)]
-    h2d = sum(t.numel() * t.element_size() for t in host_in.values())
-    d2h = sum(t.numel() * t.element_size() for t in host_out)
-    if world > 1:
-        dist.barrier()
-    torch.cuda.synchronize()
-    e0 = torch.cuda.Event(enable_timing=True)
-    e1 = torch.cuda.Event(enable_timing=True)
-    e0.record()
-    for i in range(e2e_steps):
-        for k in dev_in:
-            dev_in[k].copy_(host_in[k], non_blocking=True)
-        step(i, dev_in["W"], dev_in["X"], dev_in["A"], dev_in["B"], dev_in["dY"])
-        for h, d in zip(host_out, (Y, dX, dA, dB)):
-            h.copy_(d, non_blocking=True)
-    e1.record()
-    torch.cuda.synchronize()
-    e2e_ms = e0.elapsed_time(e1)
-    if world > 1:
-        e2e_ms = max_over_ranks(e2e_ms, dev)
-    e2e_value = whole_job_rate(flops, world, e2e_ms / e2e_steps * 1e-3) / 1e12
-
+def layer_record(name: str, ls: LayerSet, m: dict, world: int, steps: int, warmup: int) -> dict:
+    """The JSON record of one layer-set measurement (the main line's fields)."""
     hbm, bf16_burst, bf16_sus, peak_src = _peaks()
-    # dominant kernel: the fused dequant GEMM of the backward (dX) or forward (Y), whichever is longer
-    dom = "bwd_dx" if bwd_ms >= fwd_ms else "fwd_y"
-    dom_ms = max(bwd_ms, fwd_ms)
-    dom_flops = 2.0 * M * N * K + 2.0 * M * r * (K if dom == "bwd_dx" else N)
-    achieved = dom_flops / (dom_ms * 1e-3) / 1e12
-    packed = wq.nbytes()
-    traffic = None
-    if TRAFFIC_CAPTURE["sources_sha1"] and TRAFFIC_CAPTURE["sources_sha1"] == kernel_sources_sha1():
-        traffic = TRAFFIC_CAPTURE.get(dom)
-
-    line = {
+    flops = ls.flops()
+    value = whole_job_rate(flops, world, m["ms_step"] * 1e-3) / 1e12
+    ff = [fused_flops(c) for c in ls.cases]
+    fwd_f, bwd_f = sum(f for f, _ in ff), sum(b for _, b in ff)
+    fwd_t, bwd_t = sum(m["fwd_ms"]), sum(m["bwd_ms"])
+    # dominant kernel: the fused dequant GEMM variant (forward or backward) with the larger share of the step;
+    # achieved = its algorithmic flops over the seven launches / their summed event time
+    dom = "bwd" if bwd_t >= fwd_t else "fwd"
+    dom_f, dom_t = (bwd_f, bwd_t) if dom == "bwd" else (fwd_f, fwd_t)
+    achieved = dom_f / (dom_t * 1e-3) / 1e12
+    c0 = ls.cases[0]
+    batch, seq = BATCH.get(name, (1, c0.M))
+    packed = ls.packed_bytes()
+    per = [{"linear": c.name.split("_")[1] if name != "proj7b" else "proj", "N": c.N, "K": c.K,
+            "fwd_fused_ms": round(f, 5), "bwd_fused_ms": round(b, 5),
+            "fwd_fused_tflops": round(fused_flops(c)[0] / (f * 1e-3) / 1e12, 1),
+            "bwd_fused_tflops": round(fused_flops(c)[1] / (b * 1e-3) / 1e12, 1)}
+           for c, f, b in zip(ls.cases, m["fwd_ms"], m["bwd_ms"])]
+    nlin = len(ls.cases)
+    return {
         "metric": METRIC, "value": round(value, 3), "unit": "TFLOP/s", "n_gpus": world,
-        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_step, 4),
+        "steps": steps, "warmup": warmup, "ms_per_step": round(m["ms_step"], 5),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
-        "data": "synthetic (seeded numpy N(0,std) rounded to bf16)",
-        "config": {"workload": WORKLOAD, "M": M, "N": N, "K": K, "r": r, "alpha": case.alpha,
-                   "global_batch": 4 * world, "seq_len": 1024,
-                   "parallelism": (f"data parallel x{world}: a 4096-token shard per rank, dA/dB summed by one "
-                                   f"NCCL all-reduce per step" if world > 1 else "one GPU"),
-                   "step": "quantise(W) + forward + backward",
-                   "l2": f"inputs larger than L2: {NSETS} rotating input sets (W, X, dY 33.5 MB each) + 67 MB outputs"},
-        "packed_weight_gbs": round(2 * packed / (ms_step * 1e-3) / 1e9, 2),
-        "kernels": {"fwd_fused_ms": round(fwd_ms, 4), "bwd_fused_ms": round(bwd_ms, 4),
-                    "quantize_ms": round(q_ms, 4)},
-        "quantiser": {"params_per_s": round(N * K / (q_ms * 1e-3), 1),
-                      "gbs": round((2 * N * K + packed) / (q_ms * 1e-3) / 1e9, 1),
-                      "hbm_frac": round((2 * N * K + packed) / (q_ms * 1e-3) / 1e9 / hbm, 4),
-                      "bytes": "bf16 W read + stored weight written, per call (3 kernels), L2 flushed before each"},
-        "roofline": {"kernel": f"fused dequant GEMM ({dom})", "bound": "tensor",
-                     "achieved": round(achieved, 2), "peak": bf16_burst, "unit": "TFLOP/s",
-                     "frac": round(achieved / bf16_burst, 4), "peak_source": f"{peak_src} bf16 burst",
-                     "traffic": traffic, "traffic_unit": "bytes per launch (ncu dram read+write)"},
-        "e2e": {"value": round(e2e_value, 3), "unit": "TFLOP/s", "h2d_bytes_per_step": h2d,
-                "d2h_bytes_per_step": d2h, "steps": e2e_steps},
-        "gpu_launches": int(launches),
-        "clocks": clocks,
+        "data": "synthetic (seeded numpy N(0,std) rounded to bf16" +
+                ("; W with 0.1% 0.2*t(3) outliers)" if c0.outlier_frac else ")"),
+        "config": {"workload": WORKLOADS[name], "M": c0.M, "r": c0.r, "alpha": c0.alpha,
+                   "shapes": [f"{c.name.split('_')[1] if name != 'proj7b' else 'proj'} {c.N}x{c.K}"
+                              for c in ls.cases],
+                   "global_batch": batch * world, "seq_len": seq,
+                   "parallelism": (f"data parallel x{world}: a {c0.M}-token shard per rank, the adapter gradients "
+                                   f"summed by one NCCL all-reduce per step" if world > 1 else "one GPU"),
+                   "step": (f"forward of the {nlin} linears, then their backward in reverse order; the weights are "
+                            f"quantised once at load (the quantiser is reported on its own)" if nlin > 1 else
+                            "forward + backward; the weight is quantised once at load"),
+                   "l2": f"inputs larger than L2: a step reads {(packed + sum(2 * c.M * (c.K + c.N) for c in ls.cases)) / 1e9:.2f} GB"},
+        "packed_weight_gbs": round(2 * packed / (m["ms_step"] * 1e-3) / 1e9, 2),
+        "kernels": {"fwd_fused_ms": round(fwd_t, 5), "bwd_fused_ms": round(bwd_t, 5), "per_linear": per},
+        "roofline": {"kernel": f"fused dequant GEMM ({dom}, {nlin} launch{'es' if nlin > 1 else ''} per step)",
+                     "bound": "tensor", "achieved": round(achieved, 2), "peak": bf16_burst, "unit": "TFLOP/s",
+                     "frac": round(achieved / bf16_burst, 4),
+                     "frac_of_sustained": round(achieved / bf16_sus, 4) if bf16_sus else None,
+                     "peak_source": f"{peak_src} bf16 burst",
+                     "traffic": _traffic(TRAFFIC_CAPTURE, KERNEL_SOURCES, (name, dom)),
+                     "traffic_unit": f"bytes per step over the {nlin} {dom} launches (ncu dram read+write)"},
+        "e2e": {"value": round(whole_job_rate(flops, world, m["e2e_ms_step"] * 1e-3) / 1e12, 3), "unit": "TFLOP/s",
+                "h2d_bytes_per_step": m["h2d"], "d2h_bytes_per_step": m["d2h"], "steps": m["e2e_steps"]},
+        "gpu_launches": m["launches"],
+        "clocks": m["clocks"],
     }
-    if world == 1 and rank == 0 and not args.no_cpu_baseline:
-        line["cpu_baseline"] = cpu_baseline()
-    if rank == 0:
-        print(json.dumps(line), flush=True)
-    if world > 1:
-        dist.barrier()
-        dist.destroy_process_group()
 
 
-def run_smallm(args):
-    """Forward only at decode batch sizes: T = X·A, then the small-M dequant GEMM."""
+def layer_cases(name: str):
+    from bit_nf4_quantised_codebook_b200 import inputs
+    return {"shapes_65b": inputs.shapes_65b, "llama7b_layer": inputs.llama7b_layer,
+            "proj7b": lambda: [inputs.proj_7b()]}[name]()
+
+
+def measure_layer_set(name: str, steps: int, warmup: int, world: int, rank: int, local: int) -> dict:
+    import torch
+    dev = torch.device("cuda", local)
+    ls = LayerSet(layer_cases(name), dev, rank, world)
+    m = ls.measure(steps, warmup, world, local)
+    rec = layer_record(name, ls, m, world, steps, warmup)
+    del ls
+    torch.cuda.empty_cache()
+    return rec
+
+
+# ---------------------------------------------------------------- decode-sized forward
+def measure_smallm(n: int, m_tok: int, steps: int, warmup: int, world: int, local: int,
+                   e2e_steps: int | None = None) -> dict:
+    """Forward at decode batch sizes: T = X·A, then the small-M dequant GEMM.
+    The weight is quantised once and kept resident, rotated over enough copies
+    that no forward finds it in L2."""
     import torch
     import torch.distributed as dist
-    from datetime import timedelta
     from bit_nf4_quantised_codebook_b200 import api, inputs
-
-    world, rank, local = _dist()
-    torch.cuda.set_device(local)
-    if world > 1:
-        dist.init_process_group("nccl", timeout=timedelta(seconds=120), device_id=torch.device("cuda", local))
-    api.lib()
     dev = torch.device("cuda", local)
-    case = inputs.small_m(args.n, args.m)
+    case = inputs.small_m(n, m_tok)
     M, N, K, r, s = case.M, case.N, case.K, case.r, case.s
     W = api.bits_to_tensor(case.W(), dev)
     ncopy = max(2, -(-3 * 128 * 2**20 // (N * K // 2)))  # weight copies: > 3x L2 in total
@@ -394,20 +556,14 @@ def run_smallm(args):
         api.qlora_linear_forward(qs[i % ncopy], X if Xin is None else Xin, A, B, s, Y=Y, T_save=sT, ws=ws,
                                  dev_err=err)
 
-    for i in range(args.warmup):
+    for i in range(warmup):
         step(i)
     torch.cuda.synchronize()
-    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(args.steps)]
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(steps)]
     for pair in ev:
         for e in pair:
             e.record()
-    gpu_id = None
-    try:
-        gpu_id = "GPU-" + str(torch.cuda.get_device_properties(local).uuid)
-    except Exception:
-        pass
-    sampler = ClockSampler(gpu_id)
-    sampler.start()
+    sampler = _gpu_sampler(local)
     if world > 1:
         dist.barrier()
     torch.cuda.synchronize()
@@ -416,31 +572,30 @@ def run_smallm(args):
     t0 = torch.cuda.Event(enable_timing=True)
     t1 = torch.cuda.Event(enable_timing=True)
     t0.record()
-    for i in range(args.steps):
+    for i in range(steps):
         step(i)
     t1.record()
     torch.cuda.synchronize()
     sampler.mark_end()
     launches = api.qlora_kernel_launch_count() - launches0
-    # the dominant kernel alone: events around it (they end the programmatic overlap
+    # the small-M kernel alone: events around it (they end the programmatic overlap
     # with the X·A kernel, so this loop is timed separately from the step loop)
-    for i in range(args.steps):
+    for i in range(steps):
         api.qlora_set_timing_events(ev[i][0], ev[i][1])
         step(i)
     torch.cuda.synchronize()
     api.qlora_set_timing_events()
     clocks = sampler.stop()
     ms = t0.elapsed_time(t1)
-    kern_ms = sum(a.elapsed_time(b) for a, b in ev) / args.steps
+    kern_ms = sum(a.elapsed_time(b) for a, b in ev) / steps
     if world > 1:
         ms = max_over_ranks(ms, dev)
     if int(err[0].item()) != 0:
         raise RuntimeError(f"device error word {int(err[0].item())}")
-    ms_step = ms / args.steps
-    value = whole_job_rate(packed, world, ms_step * 1e-3) / 1e9
+    ms_step = ms / steps
 
     # end to end: X host -> device, forward, Y device -> host
-    e2e_steps = max(3, min(100, args.steps // 10))
+    e2e_steps = e2e_steps or max(3, min(100, steps // 10))
     hx = X.cpu().pin_memory()
     hy = torch.empty_like(Y, device="cpu").pin_memory()
     dx = torch.empty_like(X)
@@ -455,37 +610,178 @@ def run_smallm(args):
     e1.record()
     torch.cuda.synchronize()
     e2e_ms = e0.elapsed_time(e1) / e2e_steps
+    del qs
+    torch.cuda.empty_cache()
 
     hbm, _, _, peak_src = _peaks()
     achieved = packed / (kern_ms * 1e-3) / 1e9
-    line = {
-        "metric": METRIC, "value": round(value, 2), "unit": "GB/s", "n_gpus": world,
-        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_step, 5),
+    return {
+        "metric": METRIC, "value": round(whole_job_rate(packed, world, ms_step * 1e-3) / 1e9, 2), "unit": "GB/s",
+        "n_gpus": world, "steps": steps, "warmup": warmup, "ms_per_step": round(ms_step, 5),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
-        "data": "synthetic (seeded numpy N(0,std) rounded to bf16)",
+        "data": "synthetic (seeded numpy N(0,std) rounded to bf16; W with 0.1% 0.2*t(3) outliers)",
         "config": {"workload": f"small-M forward: W {N}x{K} NF4+DQ, {M} tokens, LoRA r={r} alpha={case.alpha}",
                    "M": M, "N": N, "K": K, "r": r, "parallelism": f"replicas x{world} (no shard)",
                    "step": "forward (X·A, then the dequant GEMM with the adapter term)",
                    "l2": f"{ncopy} resident weight copies used in rotation ({ncopy * packed / 1e6:.0f} MB > L2)"},
+        "packed_weight_bytes": packed,
         "kernels": {"smallm_gemm_ms": round(kern_ms, 5)},
         "roofline": {"kernel": "small-M dequant GEMM", "bound": "hbm", "achieved": round(achieved, 1),
                      "peak": hbm, "unit": "GB/s", "frac": round(achieved / hbm, 4),
                      "peak_source": f"{peak_src} HBM copy",
-                     "traffic": (SMALLM_TRAFFIC.get((N, M))
-                                 if SMALLM_TRAFFIC["sources_sha1"] == kernel_sources_sha1(SMALLM_SOURCES) else None),
+                     "traffic": _traffic(SMALLM_TRAFFIC, SMALLM_SOURCES, (N, M)),
                      "traffic_unit": "bytes per launch (ncu dram read+write)"},
         "e2e": {"value": round(packed / (e2e_ms * 1e-3) / 1e9, 2), "unit": "GB/s",
                 "h2d_bytes_per_step": X.numel() * 2, "d2h_bytes_per_step": Y.numel() * 2, "steps": e2e_steps},
         "gpu_launches": int(launches),
         "clocks": clocks,
     }
+
+
+# ---------------------------------------------------------------- quantiser (load time)
+def measure_quantiser(n: int, k: int, steps: int, local: int, w_std: float = 0.015, outliers: float = 0.001) -> dict:
+    """qlora_quantize (block kernel, mean, E4M3 constants) timed alone with events
+    around each call, a buffer larger than L2 written before each call so that W
+    comes from HBM."""
+    import torch
+    from bit_nf4_quantised_codebook_b200 import api, inputs
+    dev = torch.device("cuda", local)
+    W = api.bits_to_tensor(inputs.weight_bf16(n, k, w_std, 0, outliers), dev)
+    wq = api.alloc_weight(n, k, dev)
+    ws = torch.empty(api.qlora_workspace_size(api.QLORA_OP_QUANTIZE, 0, n, k, 0), dtype=torch.uint8, device=dev)
+    err = api.new_error_word(dev)
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    for _ in range(3):
+        api.qlora_quantize(W, out=wq, ws=ws, dev_err=err)
+    qev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
+    for i in range(steps):
+        flush.zero_()
+        qev[i][0].record()
+        api.qlora_quantize(W, out=wq, ws=ws, dev_err=err)
+        qev[i][1].record()
+    torch.cuda.synchronize()
+    if int(err[0].item()) != 0:
+        raise RuntimeError(f"device error word {int(err[0].item())}")
+    q_ms = sum(a.elapsed_time(b) for a, b in qev) / steps
+    hbm, _, _, peak_src = _peaks()
+    by = 2 * n * k + wq.nbytes()
+    del W, flush
+    torch.cuda.empty_cache()
+    return {"shape": f"{n}x{k}", "ms": round(q_ms, 5), "params_per_s": round(n * k / (q_ms * 1e-3), 1),
+            "gbs": round(by / (q_ms * 1e-3) / 1e9, 1), "hbm_frac": round(by / (q_ms * 1e-3) / 1e9 / hbm, 4),
+            "peak_source": f"{peak_src} HBM copy",
+            "bytes": "bf16 W read + stored weight written, per call (3 kernels), L2 flushed before each"}
+
+
+# ---------------------------------------------------------------- the default line
+def run_ours(args):
+    import torch
+    import torch.distributed as dist
+    from bit_nf4_quantised_codebook_b200 import api
+
+    world, rank, local = _dist()
+    _init_dist(world, local)
+    api.lib()
+    name = args.workload
+    line = measure_layer_set(name, args.steps, args.warmup, world, rank, local)
+    if name == "shapes_65b" and world == 1 and not args.no_sub:
+        sub_steps = max(args.steps, 20)
+        line["quantiser"] = measure_quantiser(22016, 8192, 20, local)
+        line["subrecords"] = {
+            "proj7b": measure_layer_set("proj7b", max(args.steps, 50), max(args.warmup, 5), 1, 0, local),
+            "llama7b_layer": measure_layer_set("llama7b_layer", sub_steps, max(args.warmup, 3), 1, 0, local),
+            "smallm": [measure_smallm(n, m, 500, 20, 1, local, e2e_steps=20)
+                       for n in (8192, 28672) for m in (1, 16)],
+        }
     if world == 1 and rank == 0 and not args.no_cpu_baseline:
-        line["cpu_baseline"] = cpu_baseline_smallm(case)
+        line["cpu_baseline"] = cpu_baseline_layers(name)
     if rank == 0:
         print(json.dumps(line), flush=True)
     if world > 1:
         dist.barrier()
         dist.destroy_process_group()
+
+
+def run_smallm(args):
+    """--workload smallm: the decode-sized forward alone."""
+    import torch.distributed as dist
+    from bit_nf4_quantised_codebook_b200 import api, inputs
+    world, rank, local = _dist()
+    _init_dist(world, local)
+    api.lib()
+    line = measure_smallm(args.n, args.m, args.steps, args.warmup, world, local)
+    if world == 1 and rank == 0 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline_smallm(inputs.small_m(args.n, args.m))
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+def cpu_baseline_smallm(case, min_seconds: float = 10.0) -> dict:
+    """The oracle on a slice of the small-M forward: quantise `rows` W rows and run
+    the forward for all tokens through them; GB/s of packed weight per host second."""
+    from oracle import linear, nf4
+    rows = 256
+    W, X, A, B = case.W()[:rows], case.X(), case.A(), case.B()[:, :rows]
+    tot_t, n = 0.0, 0
+    while tot_t < min_seconds or n == 0:
+        t = time.perf_counter()
+        what = nf4.dequantize_nf4(nf4.quantize_nf4(W))
+        linear.forward(X, what, A, B, case.s)
+        tot_t += time.perf_counter() - t
+        n += 1
+    packed = rows * case.K // 2 + rows * case.K // 64
+    return {"value": round(n * packed / tot_t / 1e9, 6), "unit": "GB/s", "cores": os.cpu_count(), "kind": "oracle",
+            "sample": f"{n} x (quantise + dequantise {rows} of the {case.N} W rows, forward for all {case.M} "
+                      f"tokens through them); {tot_t:.1f} s"}
+
+
+# ---------------------------------------------------------------- the oracle on a sample
+def oracle_sample(name: str, tok: int, wrows: int):
+    """A bounded sample of a layer set for the CPU oracle: for every linear, `tok`
+    token rows through `wrows` output features (full K, the same r, scale,
+    distributions and outliers), drawn from the workload's recipe as a layer of
+    that size.  The oracle quantises and dequantises the sample's weights
+    before the clock starts (the step keeps its weights resident too).
+    Returns (run, flops): run() is one forward + backward of every linear."""
+    from bit_nf4_quantised_codebook_b200 import inputs
+    from oracle import linear, nf4
+    prepared = {}
+    jobs = []
+    for c in layer_cases(name):
+        sc = inputs.LinearCase(c.name, tok, min(wrows, c.N), c.K, c.r, c.alpha, c.w_std, c.a_std, c.b_std,
+                               c.outlier_frac, c.seed)
+        key = (sc.N, sc.K)
+        if key not in prepared:
+            prepared[key] = (sc, nf4.dequantize_nf4(nf4.quantize_nf4(sc.W())), sc.X(), sc.A(), sc.B(), sc.dY())
+        jobs.append(prepared[key])
+    flops = sum(sc.flops_fwd() + sc.flops_bwd() for sc, *_ in jobs)
+
+    def run():
+        for sc, wh, X, A, B, dY in jobs:
+            linear.forward(X, wh, A, B, sc.s)
+            linear.backward(X, dY, wh, A, B, sc.s)
+
+    return run, flops
+
+
+def cpu_baseline_layers(name: str, min_seconds: float = 10.0) -> dict:
+    """The oracle as it stands (float64 numpy, BLAS on all host cores) on a
+    bounded sample of the layer set, repeated until `min_seconds` have passed."""
+    tok, wrows = 256, 256
+    run, flops = oracle_sample(name, tok, wrows)
+    tot_t, n = 0.0, 0
+    while tot_t < min_seconds or n == 0:
+        t = time.perf_counter()
+        run()
+        tot_t += time.perf_counter() - t
+        n += 1
+    nlin = len(layer_cases(name))
+    return {"value": round(n * flops / tot_t / 1e12, 6), "unit": "TFLOP/s", "cores": os.cpu_count(), "kind": "oracle",
+            "sample": f"{n} x fwd + bwd of the {nlin} linears on {tok} token rows through {wrows} output features "
+                      f"each (full K, r=64; float64 numpy); {tot_t:.1f} s"}
 
 
 ADAMW_SHAPES = [("q", 4096, 4096), ("k", 4096, 4096), ("v", 4096, 4096), ("o", 4096, 4096),
@@ -605,8 +901,9 @@ def run_adamw(args):
 
 
 MERGE_SHAPES = ADAMW_SHAPES  # the seven linears of one LLaMA-7B decoder layer
-# ncu DRAM read + write of the merge-and-code kernel over one step's seven launches
-# (profiles/merge_requantize_llama7b_layer.md), valid for the sources it was taken from.
+# ncu DRAM read + write of the merge-and-code kernel over one step's seven launches (a one-pass
+# `--metrics gpu__time_duration.sum,dram__bytes_read.sum,dram__bytes_write.sum -k regex:merge`
+# capture of `--workload merge`), valid for the sources it was taken from.
 MERGE_SOURCES = ["merge.cu", "nf4_decode.cuh", "nf4_quant.cuh", "ptx.cuh", "launch.cuh"]
 MERGE_TRAFFIC = {"sources_sha1": "4e714f616c7e4e56f4c0d477b522210425681dd2", "bytes_per_step": 117_096_000}
 
@@ -981,92 +1278,54 @@ def cpu_baseline_adamw(min_seconds: float = 10.0) -> dict:
             "kind": "oracle", "sample": f"{k} AdamW steps on 2^20 parameters (float64 numpy); {tot_t:.1f} s"}
 
 
-def cpu_baseline_smallm(case, min_seconds: float = 10.0) -> dict:
-    """The oracle on a slice of the small-M forward: quantise `rows` W rows and run
-    the forward for all tokens through them; GB/s of packed weight per host second."""
-    from oracle import linear, nf4
-    rows = 256
-    W, X, A, B = case.W()[:rows], case.X(), case.A(), case.B()[:, :rows]
-    tot_t, n = 0.0, 0
-    while tot_t < min_seconds or n == 0:
-        t = time.perf_counter()
-        what = nf4.dequantize_nf4(nf4.quantize_nf4(W))
-        linear.forward(X, what, A, B, case.s)
-        tot_t += time.perf_counter() - t
-        n += 1
-    packed = rows * case.K // 2 + rows * case.K // 64
-    return {"value": round(n * packed / tot_t / 1e9, 6), "unit": "GB/s", "cores": os.cpu_count(), "kind": "oracle",
-            "sample": f"{n} x (quantise + dequantise {rows} of the {case.N} W rows, forward for all {case.M} "
-                      f"tokens through them); {tot_t:.1f} s"}
-
-
-def _oracle_sample(rows: int, qrows: int | None = None):
-    """The oracle on a bounded sample of the workload: quantise + dequantise
-    `qrows` rows of the 4096 x 4096 weight (all of it by default), then forward +
-    backward for `rows` token rows through that (sub-)layer."""
-    from bit_nf4_quantised_codebook_b200 import inputs
-    from oracle import linear, nf4
-
-    case = inputs.proj_7b()
-    n = case.N if qrows is None else qrows
-    W, X, A, B, dY = case.W()[:n], case.X()[:rows], case.A(), case.B()[:, :n], case.dY()[:rows, :n]
-    t = time.perf_counter()
-    q = nf4.quantize_nf4(W)
-    what = nf4.dequantize_nf4(q)
-    linear.forward(X, what, A, B, case.s)
-    linear.backward(X, dY, what, A, B, case.s)
-    dt = time.perf_counter() - t
-    c = inputs.LinearCase(case.name, rows, n, case.K, case.r, case.alpha, case.w_std, case.a_std, case.b_std)
-    return dt, c.flops_fwd() + c.flops_bwd()
-
-
-def cpu_baseline(min_seconds: float = 10.0) -> dict:
-    """The oracle as it stands on the full workload (quantise + dequantise the
-    4096 x 4096 W, forward + backward on all 4096 token rows), repeated until
-    `min_seconds` of host time have passed."""
-    tot_t, tot_f, n = 0.0, 0.0, 0
-    while tot_t < min_seconds or n == 0:
-        dt, fl = _oracle_sample(4096)
-        tot_t += dt
-        tot_f += fl
-        n += 1
-    return {"value": round(tot_f / tot_t / 1e12, 6), "unit": "TFLOP/s", "cores": os.cpu_count(), "kind": "oracle",
-            "sample": f"{n} x the full step on the host (quantise + dequantise the 4096x4096 W, fwd + bwd on "
-                      f"4096 tokens; float64 numpy, BLAS threads = cores); {tot_t:.1f} s"}
 
 
 def run_reference(args):
-    """The oracle as the reference arm: every step is a bounded sample of the
-    workload (a slice of `n` weight rows and `n` token rows), sized so that the
-    whole --steps/--warmup run takes about two minutes of host time."""
+    """The oracle as the reference arm, on the same workload, metric and unit as
+    our line: every step is a bounded sample of the layer set (every linear,
+    `tok` token rows through `tok` output features), sized so that the whole
+    --steps/--warmup run takes about two minutes of host time.  Under torchrun
+    rank 0 alone runs it."""
     world, rank, _ = _dist()
     if rank != 0:
         return
-    # host seconds for the whole run (about two minutes; a test shortens it)
+    name = args.workload if args.workload in WORKLOADS else "shapes_65b"
     budget = float(os.environ.get("QLORA_REFERENCE_SECONDS", "120")) / max(1, args.steps + args.warmup)
     n = 16
-    dt, _ = _oracle_sample(n, n)
+    run, flops = oracle_sample(name, n, n)
+    t = time.perf_counter()
+    run()
+    dt = time.perf_counter() - t
     while n < 1024 and dt * 2.2 < budget:
         n *= 2
-        dt, _ = _oracle_sample(n, n)
+        run, flops = oracle_sample(name, n, n)
+        t = time.perf_counter()
+        run()
+        dt = time.perf_counter() - t
     for _ in range(args.warmup):
-        _oracle_sample(n, n)
-    tot_t, tot_f = 0.0, 0.0
+        run()
+    tot_t = 0.0
     for _ in range(args.steps):
-        dt, fl = _oracle_sample(n, n)
-        tot_t += dt
-        tot_f += fl
-    value = tot_f / tot_t / 1e12
+        t = time.perf_counter()
+        run()
+        tot_t += time.perf_counter() - t
+    value = args.steps * flops / tot_t / 1e12
+    cases = layer_cases(name)
+    c0 = cases[0]
+    batch, seq = BATCH[name]
+    sample = (f"per step: fwd + bwd of the {len(cases)} linears on {n} token rows through {n} output features each "
+              f"(full K, r={c0.r}), weights quantised and dequantised by the oracle before the clock starts")
     line = {
         "impl": "reference", "metric": METRIC, "value": round(value, 6), "unit": "TFLOP/s", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(tot_t / args.steps * 1e3, 3),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
         "data": "synthetic (seeded numpy N(0,std) rounded to bf16)",
-        "config": {"workload": WORKLOAD, "M": 4096, "N": 4096, "K": 4096, "r": 64, "alpha": 16.0,
-                   "global_batch": 4, "seq_len": 1024, "parallelism": "cpu oracle"},
+        "config": {"workload": WORKLOADS[name], "M": c0.M, "r": c0.r, "alpha": c0.alpha,
+                   "shapes": [f"{c.N}x{c.K}" for c in cases], "global_batch": batch, "seq_len": seq,
+                   "parallelism": "cpu oracle on the host cores (rank 0)",
+                   "sample": sample, "sample_tokens": n, "sample_output_features": n},
         "cpu_baseline": {"value": round(value, 6), "unit": "TFLOP/s", "cores": os.cpu_count(), "kind": "oracle",
-                         "sample": f"per step: quantise+dequantise {n} weight rows (K=4096), fwd+bwd on {n} "
-                                   f"token rows through them"},
+                         "sample": sample},
         "e2e": {"value": round(value, 6), "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line), flush=True)
@@ -1075,14 +1334,18 @@ def run_reference(args):
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=1000)
-    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--workload", choices=["proj7b", "smallm", "adamw", "merge", "formats"], default="proj7b")
+    ap.add_argument("--no-sub", action="store_true", help="main line only (no sub-records)")
+    ap.add_argument("--workload", choices=list(WORKLOADS) + ["smallm", "adamw", "merge", "formats"],
+                    default="shapes_65b")
     ap.add_argument("--n", type=int, default=8192, help="smallm: W rows (8192 or 28672)")
     ap.add_argument("--m", type=int, default=16, help="smallm: tokens (1..64)")
     args = ap.parse_args()
+    if args.impl == "ours":
+        args.warmup = max(3, args.warmup)  # at least three untimed steps before any timing
     if args.impl == "reference":
         run_reference(args)
     elif args.workload == "smallm":

@@ -9,11 +9,28 @@
 // dependent starts: a dependent that reads some inputs before its own wait may
 // rely on that (it must still wait before reading its predecessor's output).
 #pragma once
+#include <atomic>
+#include <cstdint>
 #include <utility>
 #include <cuda_runtime.h>
 #include "internal.h"
 
 namespace qlora {
+
+// Raises a kernel's dynamic shared-memory limit to `bytes` on the current
+// device once.  The attribute belongs to the device's context, so `done` holds
+// one bit per device (devices 64 and up set it on every call).  Two host threads
+// that race here both set the same value, which is harmless.
+inline cudaError_t smem_attr_once(const void *kern, int bytes, std::atomic<uint64_t> &done) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  const uint64_t bit = dev < 64 ? (uint64_t{1} << dev) : 0;
+  if (bit && (done.load(std::memory_order_acquire) & bit)) return cudaSuccess;
+  e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+  if (e == cudaSuccess && bit) done.fetch_or(bit, std::memory_order_acq_rel);
+  return e;
+}
 
 template <typename... KArgs, typename... Args>
 cudaError_t launch_k(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st, unsigned cz,

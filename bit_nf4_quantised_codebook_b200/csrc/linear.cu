@@ -44,11 +44,8 @@ using CfgDB = GemmCfg<BN, 4, true, B_TMA_MN, LORA_NONE, OUT_RED_F32_T>; // (dYáµ
 
 template <class C>
 static cudaError_t prepare() {
-  static bool done = false;
-  if (done) return cudaSuccess;
-  cudaError_t e = cudaFuncSetAttribute(gemm_kernel<C>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES);
-  if (e == cudaSuccess) done = true;
-  return e;
+  static std::atomic<uint64_t> done{0};
+  return smem_attr_once(reinterpret_cast<const void *>(gemm_kernel<C>), C::SMEM_BYTES, done);
 }
 
 template <class C>
@@ -75,13 +72,9 @@ constexpr int kPairTokens = 2 * 128 * 2;  // tokens per CTA pair (2 CTAs x MSUB 
 
 template <class C>
 static cudaError_t launch_pair(dim3 grid, const TmaMaps &m, const GemmParams &p, cudaStream_t st) {
-  static bool prepared = false;
-  if (!prepared) {
-    cudaError_t e = cudaFuncSetAttribute(gemm_pair_kernel<C>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         C::SMEM_BYTES);
-    if (e != cudaSuccess) return e;
-    prepared = true;
-  }
+  static std::atomic<uint64_t> prepared{0};
+  cudaError_t e = smem_attr_once(reinterpret_cast<const void *>(gemm_pair_kernel<C>), C::SMEM_BYTES, prepared);
+  if (e != cudaSuccess) return e;
   return launch_k(gemm_pair_kernel<C>, grid, dim3(C::NUM_THREADS), C::SMEM_BYTES, st, 1, m.a, m.b, m.a2, m.b2, p);
 }
 
@@ -232,13 +225,9 @@ constexpr int kSmallGroups = QLORA_SMALL_GROUPS;  // dequant groups of 4 warps p
 
 template <class C>
 static cudaError_t launch_small(dim3 grid, int cz, const TmaMaps &m, const SmallParams &p, cudaStream_t st) {
-  static bool prepared = false;
-  if (!prepared) {
-    cudaError_t e = cudaFuncSetAttribute(gemm_smallm_kernel<C>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         C::SMEM_BYTES);
-    if (e != cudaSuccess) return e;
-    prepared = true;
-  }
+  static std::atomic<uint64_t> prepared{0};
+  cudaError_t e = smem_attr_once(reinterpret_cast<const void *>(gemm_smallm_kernel<C>), C::SMEM_BYTES, prepared);
+  if (e != cudaSuccess) return e;
   return launch_k(gemm_smallm_kernel<C>, grid, dim3(C::NUM_THREADS), C::SMEM_BYTES, st, static_cast<unsigned>(cz),
                   m.a, m.b, m.a2, m.b2, p);
 }

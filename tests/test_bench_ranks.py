@@ -41,8 +41,8 @@ def test_two_rank_job_time_and_rate():
 
 
 def _dp_rank(rank: int, world: int, port: int, out):
-    """Each rank: the oracle's adapter gradients on its token shard, then the same
-    sum-all-reduce bench.py applies to its dA/dB bucket."""
+    """Each rank: the oracle's adapter gradients of two linears on its token shard,
+    written into bench.py's gradient bucket and summed by its all-reduce helper."""
     import numpy as np
     from bit_nf4_quantised_codebook_b200 import inputs
     from oracle import linear, nf4
@@ -50,28 +50,49 @@ def _dp_rank(rank: int, world: int, port: int, out):
     os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port), RANK=str(rank), WORLD_SIZE=str(world))
     dist.init_process_group("gloo", rank=rank, world_size=world)
     try:
-        case = inputs.LinearCase("dp", M=64, N=128, K=192, r=16, alpha=16.0, w_std=0.02, a_std=0.05,
-                                 b_std=0.05, seed=9)
-        what = nf4.dequantize_nf4(nf4.quantize_nf4(case.W()))
-        X, dY = case.X(), case.dY()
-        sl = slice(rank * case.M // world, (rank + 1) * case.M // world)  # this rank's token shard
-        g = linear.backward(X[sl], dY[sl], what, case.A(), case.B(), case.s)
-        bucket = torch.tensor(np.concatenate([g["dA"].ravel(), g["dB"].ravel()]))
-        dist.all_reduce(bucket)
-        full = linear.backward(X, dY, what, case.A(), case.B(), case.s)
-        out[rank] = (bucket.numpy(), np.concatenate([full["dA"].ravel(), full["dB"].ravel()]))
+        cases = [inputs.LinearCase("dp0", M=64, N=128, K=192, r=16, alpha=16.0, w_std=0.02, a_std=0.05,
+                                   b_std=0.05, seed=9),
+                 inputs.LinearCase("dp1", M=64, N=64, K=256, r=16, alpha=32.0, w_std=0.02, a_std=0.05,
+                                   b_std=0.05, seed=19)]
+        bucket, views = bench.grad_bucket([(c.K, c.r, c.N) for c in cases], torch.device("cpu"))
+        want = []
+        for c, (dA, dB) in zip(cases, views):
+            what = nf4.dequantize_nf4(nf4.quantize_nf4(c.W()))
+            X, dY = c.X(), c.dY()
+            sl = slice(rank * c.M // world, (rank + 1) * c.M // world)  # this rank's token shard
+            g = linear.backward(X[sl], dY[sl], what, c.A(), c.B(), c.s)
+            dA.copy_(torch.from_numpy(g["dA"]))
+            dB.copy_(torch.from_numpy(g["dB"]))
+            full = linear.backward(X, dY, what, c.A(), c.B(), c.s)
+            want.append((full["dA"], full["dB"]))
+        bench.allreduce_grads(bucket)
+        out[rank] = ([(dA.numpy().copy(), dB.numpy().copy()) for dA, dB in views], want)
         dist.barrier()
     finally:
         dist.destroy_process_group()
 
 
 def test_data_parallel_adapter_gradients_sum_over_shards():
-    """The exchange step of the data-parallel bench: summing the shards' dA/dB gives
-    the whole batch's gradients (they are sums over tokens)."""
+    """The exchange step of the data-parallel bench: bench.py's bucket of every
+    linear's dA/dB, summed by its all-reduce helper, holds the whole batch's
+    gradients (they are sums over tokens)."""
     world = 2
     out = mp.Manager().dict()
     mp.spawn(_dp_rank, args=(world, _free_port(), out), nprocs=world, join=True)
     for r in range(world):
-        got, full = out[r]
-        assert got.shape == full.shape
-        assert abs(got - full).max() <= 1e-12 * max(1.0, abs(full).max())
+        got, want = out[r]
+        for (ga, gb), (wa, wb) in zip(got, want):
+            assert ga.shape == wa.shape and gb.shape == wb.shape
+            for g, w in ((ga, wa), (gb, wb)):
+                assert abs(g - w).max() <= 1e-5 * max(1.0, abs(w).max())
+
+
+def test_shards_differ_by_rank():
+    """Every rank's X and dY come from their own seeds; rank 0 keeps the configuration's."""
+    from bit_nf4_quantised_codebook_b200 import inputs
+    c = inputs.LinearCase("dp", M=8, N=64, K=64, r=8, alpha=16.0, w_std=0.02, a_std=0.05, b_std=0.05, seed=3)
+    c0, c1 = bench.shard_case(c, 0), bench.shard_case(c, 1)
+    assert c0 is c
+    assert bench.tensor_key("X", c1) != bench.tensor_key("X", c0)
+    assert bench.tensor_key("dY", c1) != bench.tensor_key("dY", c0)
+    assert (c1.M, c1.N, c1.K, c1.r, c1.s) == (c.M, c.N, c.K, c.r, c.s)
