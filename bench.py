@@ -684,9 +684,10 @@ def run_ours(args):
     api.lib()
     name = args.workload
     line = measure_layer_set(name, args.steps, args.warmup, world, rank, local)
+    if name == "shapes_65b" and world == 1:
+        line["quantiser"] = measure_quantiser(22016, 8192, 20, local)
     if name == "shapes_65b" and world == 1 and not args.no_sub:
         sub_steps = max(args.steps, 20)
-        line["quantiser"] = measure_quantiser(22016, 8192, 20, local)
         line["subrecords"] = {
             "proj7b": measure_layer_set("proj7b", max(args.steps, 50), max(args.warmup, 5), 1, 0, local),
             "llama7b_layer": measure_layer_set("llama7b_layer", sub_steps, max(args.warmup, 3), 1, 0, local),

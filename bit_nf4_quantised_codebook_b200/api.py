@@ -18,6 +18,7 @@ LIB_PATH = os.path.join(_PKG, "libqlora_nf4.so")
 
 QLORA_OP_QUANTIZE, QLORA_OP_FORWARD, QLORA_OP_BACKWARD, QLORA_OP_MERGE = 0, 1, 2, 3
 QLORA_DEVERR_NONFINITE, QLORA_DEVERR_TIMEOUT = 1, 2
+QLORA_ERR_CUDA = 4
 CODEBOOKS = {"nf4": 0, "int4": 1, "fp4_e2m1": 2, "fp4_e3m0": 3}
 DQ_MODES = {"none": 0, "e4m3": 1, "int8": 2}
 
@@ -27,7 +28,7 @@ EXPORTED = [
     "qlora_kernel_launch_count", "qlora_set_timing_events", "qlora_quantize_noalloc",
     "qlora_selftest_bounded_wait", "qlora_adamw_step", "qlora_merge_requantize",
     "qlora_format_codebook", "qlora_format_sizes", "qlora_format_workspace_size", "qlora_quantize_format",
-    "qlora_dequantize_format", "qlora_quant_error",
+    "qlora_dequantize_format", "qlora_quant_error", "qlora_last_cuda_error",
 ]
 
 
@@ -90,16 +91,21 @@ def lib() -> ctypes.CDLL:
         L.qlora_quant_error.argtypes = [vp, vp, i64, vp, vp]
         L.qlora_merge_requantize.argtypes = [ctypes.POINTER(_Weight), vp, vp, i32, f32, ctypes.POINTER(_Weight),
                                              vp, vp, sz, vp, vp]
+        L.qlora_last_cuda_error.argtypes = [vp]
         for name in EXPORTED[1:]:
-            if name != "qlora_kernel_launch_count":
+            if name not in ("qlora_kernel_launch_count", "qlora_last_cuda_error"):
                 getattr(L, name).restype = i32
+        L.qlora_last_cuda_error.restype = ctypes.c_char_p
         _lib = L
     return _lib
 
 
 def _check(st: int, what: str) -> None:
     if st != 0:
-        raise QloraError(f"{what}: {lib().qlora_status_string(st).decode()} (status {st})")
+        msg = f"{what}: {lib().qlora_status_string(st).decode()} (status {st})"
+        if st == QLORA_ERR_CUDA:
+            msg += f": {lib().qlora_last_cuda_error(None).decode()}"
+        raise QloraError(msg)
 
 
 def _ptr(t: torch.Tensor | None) -> int | None:

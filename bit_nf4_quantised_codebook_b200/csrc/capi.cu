@@ -152,6 +152,14 @@ TimingHooks g_hooks;
 
 }  // namespace
 
+thread_local int t_last_cuda_error = 0;
+
+qlora_status cuda_status(cudaError_t e) {
+  if (e == cudaSuccess) return QLORA_OK;
+  t_last_cuda_error = static_cast<int>(e);
+  return QLORA_ERR_CUDA;
+}
+
 void count_launches(int n) { g_launches.fetch_add(static_cast<uint64_t>(n), std::memory_order_relaxed); }
 const TimingHooks &timing_hooks() { return g_hooks; }
 
@@ -211,7 +219,8 @@ bool map_bf16_mn(CUtensorMap *m, const void *ptr, int64_t inner, int64_t outer) 
 }
 bool map_codes(CUtensorMap *m, const void *codes, int64_t N, int64_t K, int box_bytes, int box_rows,
                int swizzle_bytes) {
-  const CUtensorMapSwizzle sw = swizzle_bytes == 64   ? CU_TENSOR_MAP_SWIZZLE_64B
+  const CUtensorMapSwizzle sw = swizzle_bytes == 128  ? CU_TENSOR_MAP_SWIZZLE_128B
+                                : swizzle_bytes == 64 ? CU_TENSOR_MAP_SWIZZLE_64B
                                 : swizzle_bytes == 32 ? CU_TENSOR_MAP_SWIZZLE_32B
                                                       : CU_TENSOR_MAP_SWIZZLE_NONE;
   return encode_2d(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, codes, K / 2, N, K / 2, box_bytes, box_rows, sw);
@@ -222,6 +231,11 @@ bool map_codes(CUtensorMap *m, const void *codes, int64_t N, int64_t K, int box_
 using namespace qlora;
 
 extern "C" {
+
+const char *qlora_last_cuda_error(int *code) {
+  if (code) *code = t_last_cuda_error;
+  return t_last_cuda_error ? cudaGetErrorString(static_cast<cudaError_t>(t_last_cuda_error)) : "no error";
+}
 
 const char *qlora_status_string(qlora_status st) {
   switch (st) {
@@ -283,7 +297,7 @@ qlora_status qlora_quantize(const uint16_t *W, const qlora_nf4_weight *out, void
                                   reinterpret_cast<float *>(w8 + pl.off_absmax),
                                   reinterpret_cast<double *>(w8 + pl.off_gsum), pl.gsum_size, thr, dev_err,
                                   static_cast<cudaStream_t>(stream));
-  return e == cudaSuccess ? QLORA_OK : QLORA_ERR_CUDA;
+  return cuda_status(e);
 }
 
 qlora_status qlora_dequantize(const qlora_nf4_weight *w, uint16_t *W_out, void *stream) {
@@ -297,7 +311,7 @@ qlora_status qlora_dequantize(const qlora_nf4_weight *w, uint16_t *W_out, void *
   std::memcpy(lv.q, g.levels, sizeof(lv.q));
   cudaError_t e = launch_dequantize(w->codes, w->c2q, w->c1, w->mean, w->N * w->K / 64, lv, W_out,
                                     static_cast<cudaStream_t>(stream));
-  return e == cudaSuccess ? QLORA_OK : QLORA_ERR_CUDA;
+  return cuda_status(e);
 }
 
 // True when [a, a+na) and [b, b+nb) share a byte.
@@ -343,7 +357,7 @@ qlora_status qlora_merge_requantize(const qlora_nf4_weight *w, const uint16_t *A
                                                 reinterpret_cast<float *>(w8 + pl.off_absmax),
                                                 reinterpret_cast<double *>(w8 + pl.off_gsum), pl.gsum_size, lv, thr,
                                                 dev_err, g.timeout_ns, static_cast<cudaStream_t>(stream));
-  return e == cudaSuccess ? QLORA_OK : QLORA_ERR_CUDA;
+  return cuda_status(e);
 }
 
 // ---------------------------------------------------------------- format variants
@@ -429,7 +443,7 @@ qlora_status qlora_quantize_format(const uint16_t *W, const qlora_qweight *w, vo
   const cudaError_t e = launch_quantize_format(W, *w, levels, thr, reinterpret_cast<float *>(w8),
                                                reinterpret_cast<double *>(w8 + off_gsum), gsum_size, dev_err,
                                                static_cast<cudaStream_t>(stream));
-  return e == cudaSuccess ? QLORA_OK : QLORA_ERR_CUDA;
+  return cuda_status(e);
 }
 
 qlora_status qlora_dequantize_format(const qlora_qweight *w, uint16_t *W_out, void *stream) {
@@ -441,7 +455,7 @@ qlora_status qlora_dequantize_format(const qlora_qweight *w, uint16_t *W_out, vo
   float levels[16];
   build_format_codebook_f32(w->fmt.codebook, levels, nullptr);
   const cudaError_t e = launch_dequantize_format(*w, levels, W_out, static_cast<cudaStream_t>(stream));
-  return e == cudaSuccess ? QLORA_OK : QLORA_ERR_CUDA;
+  return cuda_status(e);
 }
 
 qlora_status qlora_quant_error(const uint16_t *W, const uint16_t *W_hat, int64_t n, double *stats, void *stream) {
@@ -450,7 +464,7 @@ qlora_status qlora_quant_error(const uint16_t *W, const uint16_t *W_hat, int64_t
     return QLORA_ERR_MISALIGNED;
   if (!device_ok()) return QLORA_ERR_NO_DEVICE;
   const cudaError_t e = launch_quant_error(W, W_hat, n, stats, device_sms(), static_cast<cudaStream_t>(stream));
-  return e == cudaSuccess ? QLORA_OK : QLORA_ERR_CUDA;
+  return cuda_status(e);
 }
 
 static LaunchCtx make_ctx(int *dev_err, void *stream) {
@@ -477,7 +491,7 @@ qlora_status qlora_linear_forward(const qlora_nf4_weight *w, const uint16_t *X, 
   if (!aligned16(ws)) return QLORA_ERR_MISALIGNED;
   cudaError_t e = run_forward(make_ctx(dev_err, stream), *w, X, M, A, B, r, s, Y, T_save, pl,
                               static_cast<uint8_t *>(ws));
-  return e == cudaSuccess ? QLORA_OK : QLORA_ERR_CUDA;
+  return cuda_status(e);
 }
 
 qlora_status qlora_linear_backward(const qlora_nf4_weight *w, const uint16_t *X, const uint16_t *dY, int64_t M,
@@ -496,7 +510,7 @@ qlora_status qlora_linear_backward(const qlora_nf4_weight *w, const uint16_t *X,
   if (!aligned16(ws)) return QLORA_ERR_MISALIGNED;
   cudaError_t e = run_backward(make_ctx(dev_err, stream), *w, X, dY, M, A, B, r, s, T_saved, dX, dA, dB, pl,
                                static_cast<uint8_t *>(ws));
-  return e == cudaSuccess ? QLORA_OK : QLORA_ERR_CUDA;
+  return cuda_status(e);
 }
 
 uint64_t qlora_kernel_launch_count(void) { return g_launches.load(std::memory_order_relaxed); }
@@ -520,7 +534,7 @@ qlora_status qlora_adamw_step(const qlora_adamw_tensor *tensors, int count, floa
   if (!(bc1 > 0.0) || !(bc2 > 0.0)) return QLORA_ERR_INVALID_ARG;
   cudaError_t e = launch_adamw(tensors, count, lr, beta1, beta2, eps, weight_decay, static_cast<double>(lr) / bc1,
                                std::sqrt(bc2), device_sms(), static_cast<cudaStream_t>(stream));
-  return e == cudaSuccess ? QLORA_OK : QLORA_ERR_CUDA;
+  return cuda_status(e);
 }
 
 qlora_status qlora_selftest_bounded_wait(unsigned timeout_us, int *dev_err, int *gave_up, void *stream) {
@@ -528,7 +542,7 @@ qlora_status qlora_selftest_bounded_wait(unsigned timeout_us, int *dev_err, int 
   if (!device_ok()) return QLORA_ERR_NO_DEVICE;
   cudaError_t e = launch_selftest_wait(static_cast<unsigned long long>(timeout_us) * 1000ull, dev_err, gave_up,
                                        static_cast<cudaStream_t>(stream));
-  return e == cudaSuccess ? QLORA_OK : QLORA_ERR_CUDA;
+  return cuda_status(e);
 }
 
 qlora_status qlora_set_timing_events(void *fwd_begin, void *fwd_end, void *bwd_begin, void *bwd_end) {

@@ -15,6 +15,9 @@ struct Nf4Thresholds {
 
 // Process-wide diagnostics (capi.cu).
 void count_launches(int n);
+// QLORA_OK for cudaSuccess; otherwise records `e` as this host thread's last CUDA
+// failure (qlora_last_cuda_error) and returns QLORA_ERR_CUDA.
+qlora_status cuda_status(cudaError_t e);
 struct TimingHooks {
   cudaEvent_t fwd_begin = nullptr, fwd_end = nullptr, bwd_begin = nullptr, bwd_end = nullptr;
 };

@@ -56,7 +56,10 @@ cudaError_t launch_k(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem,
   cfg.numAttrs = n;
   const cudaError_t e = cudaLaunchKernelEx(&cfg, kern, std::forward<Args>(args)...);
   count_launches(1);
-  return e != cudaSuccess ? e : cudaGetLastError();
+  // consume the launch's error state either way, so that a failed launch is not
+  // reported again by the next one
+  const cudaError_t last = cudaGetLastError();
+  return e != cudaSuccess ? e : last;
 }
 
 }  // namespace qlora

@@ -51,7 +51,8 @@ LinearPlan make_plan(int op, int64_t M, int64_t N, int64_t K, int r, int num_sms
 bool map_bf16_kmajor(CUtensorMap *m, const void *ptr, int64_t inner, int64_t outer, int box_rows);
 // bf16 [outer, inner] row-major, read MN-major (inner = MN): box {64, 64}, 128-byte swizzle.
 bool map_bf16_mn(CUtensorMap *m, const void *ptr, int64_t inner, int64_t outer);
-// packed codes of an N x K weight, uint8 [N, K/2]: box {box_bytes, box_rows}; swizzle_bytes 0 (none), 32 or 64.
+// packed codes of an N x K weight, uint8 [N, K/2]: box {box_bytes, box_rows}; swizzle_bytes 0 (none), 32, 64
+// or 128.
 bool map_codes(CUtensorMap *m, const void *codes, int64_t N, int64_t K, int box_bytes, int box_rows,
                int swizzle_bytes);
 

@@ -80,6 +80,38 @@ __device__ __forceinline__ uint32_t nf4_code(float xh, const Thresholds &t) {
 // path (exact there: see quotient_rn); smaller ones divide directly.
 constexpr float kFastQuotientMinAbsmax = 7.888609052210118e-31f;  // 2^-100
 
+// Centred buckets, for an index computed without a float-to-int conversion:
+// v = x_hat * 32 + 32 + 2^23, one fused multiply-add rounded to nearest, holds
+// round(x_hat * 32 + 32) in its low mantissa bits (0 .. 64 for x_hat in
+// [-1, 1]).  Bucket b therefore covers x_hat in [(b - 1/2)/32 - 1,
+// (b + 1/2)/32 - 1], widened by the same margin on each side, which again holds
+// at most one threshold (width 1/32 + 2/1024 < 0.0796).  65 buckets.
+constexpr int kCentredBuckets = 65;
+constexpr float kCentredMagic = 8388608.0f + 32.0f;  // 2^23 + 32: exact in float32
+constexpr int kCentredMagicBits = 0x4B000020;        // its bit pattern
+
+__device__ __forceinline__ CodeBucket make_bucket_centred(int b, const float (&t)[15]) {
+  const float lo = (static_cast<float>(b) - 0.5f) / kBucketScale - 1.0f - kBucketMargin;
+  const float hi = (static_cast<float>(b) + 0.5f) / kBucketScale - 1.0f + kBucketMargin;
+  CodeBucket e;
+  e.base = 0;
+  e.thr = __int_as_float(0x7F800000);  // +inf
+#pragma unroll
+  for (int i = 0; i < 15; ++i) {
+    if (t[i] < lo) e.base += 1;
+    else if (t[i] <= hi) e.thr = t[i];
+  }
+  return e;
+}
+
+// Code of x_hat in [-1, 1] from a centred table replicated once per lane
+// ([bucket][lane], so 32 lanes with arbitrary buckets never share a bank).
+__device__ __forceinline__ uint32_t lane_centred_code(float xh, const CodeBucket (*tab)[32], int lane) {
+  const int b = __float_as_int(__fmaf_rn(xh, kBucketScale, kCentredMagic)) - (kCentredMagicBits - 32);
+  const CodeBucket e = tab[b][lane];
+  return static_cast<uint32_t>(e.base + (xh >= e.thr ? 1 : 0));
+}
+
 // Same lookup in a table replicated once per lane ([bucket][lane]), so that 32
 // lanes looking up arbitrary buckets never share a bank.
 __device__ __forceinline__ uint32_t lane_bucket_code(float xh, const CodeBucket (*tab)[32], int lane) {

@@ -64,41 +64,91 @@ __device__ __forceinline__ double tree_sum256(double *s) {
   return v;
 }
 
-// One CTA walks groups g = blockIdx.x, blockIdx.x + gridDim.x, ...; while it
-// codes one group the 16-byte loads of its next group are already in flight.
-__global__ void __launch_bounds__(256, 2) k_quant_blocks(const uint16_t *__restrict__ W, int64_t nb,
-                                                          uint8_t *__restrict__ codes, float *__restrict__ absmax,
-                                                          double *__restrict__ gsum, Nf4Thresholds thr,
-                                                          int *dev_err) {
-  __shared__ double s_sum[256];
-  __shared__ CodeBucket s_tab[kBuckets][32];  // one copy per lane: conflict-free random lookups
-  for (int i = threadIdx.x; i < kBuckets * 32; i += 256) s_tab[i >> 5][i & 31] = make_bucket(i >> 5, thr.t);
+// 1-D bulk copy (TMA, no tensor map) of `bytes` (a multiple of 16, both addresses
+// 16-byte aligned) from global to this CTA's shared memory, completing on `bar`.
+__device__ __forceinline__ void bulk_load(void *dst, const void *src, uint32_t bytes, uint64_t *bar) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+          smem_u32(dst)),
+      "l"(src), "r"(bytes), "r"(smem_u32(bar))
+      : "memory");
+}
+
+constexpr unsigned long long kQuantWaitNs = 2000000000ull;  // bound on a wait for a group's bytes (2 s)
+constexpr int kQThreads = 1024;                   // 32 warps; 8 threads per 64-element block
+constexpr int kQStages = 4;                       // groups in the shared-memory ring
+constexpr int kQGroupBytes = 256 * 64 * 2;        // one group of 256 blocks of bfloat16: 32 KiB
+constexpr int kQTabBytes = kCentredBuckets * 32 * static_cast<int>(sizeof(CodeBucket));
+constexpr int kQSmemBytes = kQStages * kQGroupBytes + kQTabBytes + 2 * 256 * 8 + kQStages * 8 + 128;
+
+// One CTA of 1024 threads per SM walks groups g = blockIdx.x, blockIdx.x +
+// gridDim.x, ...  Each group's 32 KiB of bfloat16 weights arrive in a 4-deep
+// shared-memory ring by one bulk copy, issued three groups ahead, so HBM reads
+// never wait on the arithmetic.  Eight threads share a block: 16-byte chunk each, absmax by three
+// xor-shuffles, exact quotient and code (nf4_quant.cuh), nibble packing.  The
+// group's 256 absmax values are summed by one warp in the pairwise-tree order
+// (a[i] += a[i + h] for h = 128 .. 1) while the other warps start the next group.
+__global__ void __launch_bounds__(kQThreads, 1) k_quant_blocks(const uint16_t *__restrict__ W, int64_t nb,
+                                                                uint8_t *__restrict__ codes,
+                                                                float *__restrict__ absmax, double *__restrict__ gsum,
+                                                                Nf4Thresholds thr, int *dev_err,
+                                                                unsigned long long timeout_ns) {
+  extern __shared__ __align__(128) uint8_t q_smem[];
+  uint8_t *ring = q_smem;
+  CodeBucket(*tab)[32] = reinterpret_cast<CodeBucket(*)[32]>(q_smem + kQStages * kQGroupBytes);
+  double *s_amax = reinterpret_cast<double *>(q_smem + kQStages * kQGroupBytes + kQTabBytes);  // [2][256]
+  uint64_t *full = reinterpret_cast<uint64_t *>(s_amax + 2 * 256);
+  volatile int *abort_flag = reinterpret_cast<volatile int *>(full + kQStages);
+  const int tid = threadIdx.x;
+  const int lane = tid & 31;
+  const int part = tid & 7;  // 8-element chunk of the block
   const int64_t ng = (nb + 255) / 256;
-  const int part = threadIdx.x & 7;  // 8-element chunk of the block
-  const int sub = threadIdx.x >> 3;  // block within the pass
-  const int lane = threadIdx.x & 31;
-  auto load_group = [&](int64_t g, uint4 (&raw)[8]) {
-#pragma unroll
-    for (int pass = 0; pass < 8; ++pass) {
-      const int64_t b = g * 256 + pass * 32 + sub;
-      raw[pass] = (g < ng && b < nb) ? ld_stream_v4(W + b * 64 + part * 8) : make_uint4(0, 0, 0, 0);
-    }
-  };
+  for (int i = tid; i < kCentredBuckets * 32; i += kQThreads) tab[i >> 5][i & 31] = make_bucket_centred(i >> 5, thr.t);
+  if (tid == 0) {
+    for (int s = 0; s < kQStages; ++s) mbar_init(&full[s], 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  __syncthreads();
   pdl_wait();
   pdl_launch_dependents();
-  uint4 cur[8], nxt[8];
-  int64_t g = blockIdx.x;
-  load_group(g, cur);
-  __syncthreads();  // bucket table ready
+  auto issue = [&](int64_t g, int s) {
+    const int64_t blocks = nb - g * 256 < 256 ? nb - g * 256 : 256;
+    const uint32_t bytes = static_cast<uint32_t>(blocks) * 128;
+    mbar_arrive_expect_tx(&full[s], bytes);
+    bulk_load(ring + s * kQGroupBytes, W + g * 256 * 64, bytes, &full[s]);
+  };
+  int issued = 0;  // groups issued (thread 0), group k of this CTA into stage k % kQStages
+  if (tid == 0)
+    for (int k = 0; k < kQStages - 1; ++k) {
+      const int64_t g = blockIdx.x + static_cast<int64_t>(k) * gridDim.x;
+      if (g < ng) {
+        issue(g, k);
+        ++issued;
+      }
+    }
   bool bad = false;
-  for (; g < ng; g += gridDim.x) {
-    load_group(g + gridDim.x, nxt);
+  int it = 0;
+  for (int64_t g = blockIdx.x; g < ng; g += gridDim.x, ++it) {
+    const int s = it % kQStages;
+    if (tid == 0) {  // the stage freed at the end of the previous group takes the group three ahead
+      const int64_t g2 = g + static_cast<int64_t>(kQStages - 1) * gridDim.x;
+      if (g2 < ng) {
+        issue(g2, (it + kQStages - 1) % kQStages);
+        ++issued;
+      }
+    }
+    const bool ok = mbar_wait_bounded(&full[s], (it / kQStages) & 1, abort_flag, dev_err, timeout_ns);
+    if (__syncthreads_or(!ok)) break;
+    const uint8_t *st = ring + s * kQGroupBytes;
+    double *sa = s_amax + (it & 1) * 256;
 #pragma unroll
-    for (int pass = 0; pass < 8; ++pass) {
-      const int lb = pass * 32 + sub;
+    for (int pass = 0; pass < 256 * 8 / kQThreads; ++pass) {
+      const int lb = pass * (kQThreads / 8) + (tid >> 3);  // block within the group
       const int64_t b = g * 256 + lb;
       const bool valid = b < nb;
-      const uint32_t u[4] = {cur[pass].x, cur[pass].y, cur[pass].z, cur[pass].w};
+      uint32_t u[4] = {0, 0, 0, 0};
+      if (valid) ld_shared_v4(smem_u32(st + lb * 128 + part * 16), u[0], u[1], u[2], u[3]);
       float x[8];
 #pragma unroll
       for (int i = 0; i < 4; ++i) {
@@ -121,10 +171,8 @@ __global__ void __launch_bounds__(256, 2) k_quant_blocks(const uint16_t *__restr
         packed = 0;
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
-          const float xa = quotient_rn(x[2 * i], amax, ra);
-          const float xb = quotient_rn(x[2 * i + 1], amax, ra);
-          const uint32_t hi = lane_bucket_code(xa, s_tab, lane);
-          const uint32_t lo = lane_bucket_code(xb, s_tab, lane);
+          const uint32_t hi = lane_centred_code(quotient_rn(x[2 * i], amax, ra), tab, lane);
+          const uint32_t lo = lane_centred_code(quotient_rn(x[2 * i + 1], amax, ra), tab, lane);
           packed |= ((hi << 4) | lo) << (8 * i);
         }
       } else if (amax > 0.f) {
@@ -140,15 +188,34 @@ __global__ void __launch_bounds__(256, 2) k_quant_blocks(const uint16_t *__restr
         reinterpret_cast<uint32_t *>(codes + b * 32)[part] = packed;
         if (part == 0) absmax[b] = amax;
       }
-      if (part == 0) s_sum[lb] = valid ? static_cast<double>(amax) : 0.0;
+      if (part == 0) sa[lb] = valid ? static_cast<double>(amax) : 0.0;
     }
-    // group sum: pairwise tree over the 256 (zero-padded) block constants
-    const double gs = tree_sum256(s_sum);
-    if (threadIdx.x == 0) gsum[g] = gs;
-    __syncthreads();  // s_sum is reused by the next group
+    __syncthreads();  // the stage is free again; the group's absmax values are in sa
+    if (tid < 32) {
+      // pairwise tree over the 256 (zero-padded) block constants: lane l holds
+      // a[l + 32j]; h = 128, 64, 32 in registers, then h = 16 .. 1 across lanes
+      double v[8];
 #pragma unroll
-    for (int pass = 0; pass < 8; ++pass) cur[pass] = nxt[pass];
+      for (int j = 0; j < 8; ++j) v[j] = sa[lane + 32 * j];
+#pragma unroll
+      for (int j = 0; j < 4; ++j) v[j] = __dadd_rn(v[j], v[j + 4]);
+#pragma unroll
+      for (int j = 0; j < 2; ++j) v[j] = __dadd_rn(v[j], v[j + 2]);
+      double a = __dadd_rn(v[0], v[1]);
+#pragma unroll
+      for (int h = 16; h >= 1; h >>= 1) {
+        const double o = __shfl_down_sync(0xFFFFFFFFu, a, h);
+        if (lane < h) a = __dadd_rn(a, o);
+      }
+      if (lane == 0) gsum[g] = a;
+    }
   }
+  // groups issued but never consumed (only after an abort) land before the CTA exits
+  if (tid == 0)
+    for (int k = it; k < issued; ++k) {
+      int dummy = 0;
+      mbar_wait_bounded(&full[k % kQStages], (k / kQStages) & 1, &dummy, nullptr, kQuantWaitNs);
+    }
   if (bad && dev_err) atomicOr(dev_err, QLORA_DEVERR_NONFINITE);
 }
 
@@ -254,9 +321,12 @@ cudaError_t launch_quantize(const uint16_t *W, int64_t nb, uint8_t *codes, uint8
   const int64_t ng = (nb + 255) / 256;
   int dev = 0, sms = 148;
   if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-  const int64_t grid = ng < 2 * static_cast<int64_t>(sms) ? ng : 2 * static_cast<int64_t>(sms);
-  cudaError_t e = launch_k(k_quant_blocks, dim3(static_cast<unsigned>(grid)), dim3(256), 0, st, 1, W, nb, codes,
-                           ws_absmax, ws_gsum, thr, dev_err);
+  const int64_t grid = ng < static_cast<int64_t>(sms) ? ng : static_cast<int64_t>(sms);
+  static std::atomic<uint64_t> prepared{0};
+  cudaError_t e = smem_attr_once(reinterpret_cast<const void *>(k_quant_blocks), kQSmemBytes, prepared);
+  if (e != cudaSuccess) return e;
+  e = launch_k(k_quant_blocks, dim3(static_cast<unsigned>(grid)), dim3(kQThreads), kQSmemBytes, st, 1, W, nb, codes,
+               ws_absmax, ws_gsum, thr, dev_err, kQuantWaitNs);
   if (e != cudaSuccess) return e;
   return launch_mean_and_double_quant(ws_absmax, nb, ws_gsum, gsum_size, mean, c2q, c1, st);
 }

@@ -23,9 +23,14 @@
 // of the mean's summation tree is cleared by the kernel that reads it).
 //
 // Host code cannot use the array's name as a device address (it is a host-side
-// stand-in for the symbol), so the first call on each device, with that device
-// current, looks the address up with cudaGetSymbolAddress and caches it; that
-// first call should therefore be made before any stream capture begins.
+// stand-in for the symbol), so each call looks the address up with
+// cudaGetSymbolAddress on the current device and remembers it per device.  A
+// call made while its stream is being captured into a CUDA graph uses the
+// remembered address instead (looking a symbol up can load the module, which
+// capture does not allow), so the first call on each device should come before
+// any stream capture.  Looking the address up again on every other call keeps it
+// valid after cudaDeviceReset or a new primary context, which reload the module
+// at another address.
 #include <cstdint>
 #include <cstring>
 #include <mutex>
@@ -49,18 +54,24 @@ constexpr int kMaxDevices = 64;
 std::mutex g_mu;
 void *g_scratch_ptr[kMaxDevices] = {};
 
-// Device address of g_quant_scratch on the current device (looked up once per device).
-cudaError_t scratch_for_current_device(void **out) {
+// Device address of g_quant_scratch on the current device: looked up afresh unless
+// `stream` is capturing, when the address remembered from an earlier call is used.
+cudaError_t scratch_for_current_device(cudaStream_t stream, void **out) {
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
   if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+  cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
+  e = cudaStreamIsCapturing(stream, &cs);
+  if (e != cudaSuccess) return e;
   std::lock_guard<std::mutex> lock(g_mu);
-  if (!g_scratch_ptr[dev]) {
+  if (cs == cudaStreamCaptureStatusNone) {
     void *p = nullptr;
     e = cudaGetSymbolAddress(&p, g_quant_scratch);
     if (e != cudaSuccess) return e;
     g_scratch_ptr[dev] = p;
+  } else if (!g_scratch_ptr[dev]) {
+    return cudaErrorStreamCaptureUnsupported;  // no earlier call on this device to take the address from
   }
   *out = g_scratch_ptr[dev];
   return cudaSuccess;
@@ -87,7 +98,8 @@ extern "C" qlora_status qlora_quantize_noalloc(const uint16_t *W, const qlora_nf
       cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess || major != 10)
     return QLORA_ERR_NO_DEVICE;
   void *scratch = nullptr;
-  if (scratch_for_current_device(&scratch) != cudaSuccess) return QLORA_ERR_CUDA;
+  const cudaError_t es = scratch_for_current_device(static_cast<cudaStream_t>(stream), &scratch);
+  if (es != cudaSuccess) return cuda_status(es);
   float levels[16];
   Nf4Thresholds thr;
   build_codebook_f32(levels, thr.t);
@@ -100,5 +112,5 @@ extern "C" qlora_status qlora_quantize_noalloc(const uint16_t *W, const qlora_nf
       launch_quantize(W, nb, out->codes, out->c2q, out->c1, out->mean, reinterpret_cast<float *>(base),
                       reinterpret_cast<double *>(base + kAbsmaxBytes), tree, thr, dev_err,
                       static_cast<cudaStream_t>(stream));
-  return e == cudaSuccess ? QLORA_OK : QLORA_ERR_CUDA;
+  return cuda_status(e);
 }

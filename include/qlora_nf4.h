@@ -91,6 +91,14 @@ enum { QLORA_OP_QUANTIZE = 0, QLORA_OP_FORWARD = 1, QLORA_OP_BACKWARD = 2, QLORA
 const char *qlora_status_string(qlora_status st);
 
 /*
+ * Diagnostic with no counterpart on the pages: the CUDA runtime's message
+ * (static string) for the last CUDA failure that made a call on this host
+ * thread return QLORA_ERR_CUDA, or "no error"; *code (nullable) receives its
+ * cudaError_t value (0 when none).
+ */
+const char *qlora_last_cuda_error(int *code);
+
+/*
  * qlora_build_codebook — host only.  §NormalFloat (intuitivepapers.ai): the
  * offset recipe (tail probability 0.9677083; 8 positive normal quantiles at
  * probabilities evenly spaced from the offset towards 1/2, 7 negative ones
@@ -146,8 +154,12 @@ qlora_status qlora_quantize(const uint16_t *W, const qlora_nf4_weight *out, void
  * calls no cudaMalloc, cudaFree or allocating routine.
  * Limit: N*K <= 2^26 (e.g. 8192 x 8192); larger weights return
  * QLORA_ERR_TOO_LARGE and launch nothing.
- * The first call on each device (with that device current) looks up the
- * array's device address; make that first call before any stream capture.
+ * Each call looks up the array's device address on the current device; a call
+ * on a stream that is being captured uses the address remembered from an
+ * earlier call on that device instead (and fails with QLORA_ERR_CUDA if there
+ * was none), so make the first call on each device before any stream capture.
+ * The lookup on every other call keeps the address right after cudaDeviceReset
+ * or a new primary context, which reload the library's module elsewhere.
  * All calls share the array: calls that overlap on the GPU (different
  * streams or host threads) race and give undefined results; calls ordered on
  * one stream are safe.  The array keeps the last call's contents; nothing in it

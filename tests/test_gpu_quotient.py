@@ -4,7 +4,8 @@ The quantiser normalises each weight by its block absmax with one reciprocal
 per block and a corrected quotient per element, and finds the code from a
 bucket table (csrc/nf4_quant.cuh).  tests/cuda/check_quotient.cu runs both
 over every bfloat16 pair (x, a) the fast path can meet and compares against
-CUDA's correctly rounded division and a plain threshold count: the codes must
+CUDA's correctly rounded division and a plain threshold count: the codes (from
+the floor-indexed table and from the centred table the quantiser uses) must
 agree for every pair and the quotients bit for bit wherever they can matter.
 """
 import os
@@ -35,3 +36,4 @@ def test_fast_quotient_and_bucket_code_exhaustive():
     assert int(fields["pairs"]) > 10 ** 9
     assert int(fields["bad_code"]) == 0, out.stdout
     assert int(fields["bad_quotient"]) == 0, out.stdout
+    assert int(fields["bad_centred"]) == 0, out.stdout
