@@ -75,11 +75,17 @@ def _peaks():
 # kernels, from one-pass ncu launch-list captures, reported only while the kernel
 # sources hash to the build each capture was taken of (otherwise null).
 # Fused dequant GEMMs: `ncu --metrics gpu__time_duration.sum,dram__bytes_read.sum,
-# dram__bytes_write.sum --clock-control none -k regex:gemm_pair` over one step of
-# each layer set; bytes per step summed over the seven forward (fwd) or backward
-# (bwd) launches.
+# dram__bytes_write.sum --clock-control none -s 147 -c 42` over one step of the
+# LLaMA-7B layer set (`--workload llama7b_layer --steps 3 --warmup 3`); bytes per step
+# summed over the seven forward (fwd) or backward (bwd) launches.  The 65B set holds
+# about 5.5 GB on the device, more than a multi-metric capture should save and
+# restore, so its figures are the LLaMA capture's traffic per algorithmic byte
+# (0.842 fwd, 1.006 bwd) times the 65B launches' algorithmic bytes.
 KERNEL_SOURCES = ["gemm_pair.cuh", "gemm.cuh", "nf4_decode.cuh", "ptx.cuh", "launch.cuh", "linear.cu"]
-TRAFFIC_CAPTURE = {"sources_sha1": None}
+TRAFFIC_CAPTURE = {"sources_sha1": "b5144ea8dd10c7c950961b46652a80443e011c46",
+                   ("llama7b_layer", "fwd"): 634_221_568, ("llama7b_layer", "bwd"): 756_754_944,
+                   ("shapes_65b", "fwd"): 2_521_543_917, ("shapes_65b", "bwd"): 3_010_471_761}
+TRAFFIC_SCALED = {"shapes_65b"}
 # The small-M kernel: the same one-pass capture of `--workload smallm`, bytes per launch, per (N, M).
 SMALLM_SOURCES = ["gemm_smallm.cuh", "gemm.cuh", "nf4_decode.cuh", "ptx.cuh", "launch.cuh", "linear.cu"]
 SMALLM_TRAFFIC = {"sources_sha1": None}
@@ -285,6 +291,16 @@ def shard_case(c, rank: int):
     from bit_nf4_quantised_codebook_b200 import inputs
     return c if rank == 0 else inputs.LinearCase(c.name, c.M, c.N, c.K, c.r, c.alpha, c.w_std, c.a_std, c.b_std,
                                                  c.outlier_frac, c.seed + 1000 * rank)
+
+
+def fused_bytes(c) -> tuple[int, int]:
+    """Algorithmic bytes of the two fused dequant GEMM launches of one linear: the
+    activation read, the stored weight read once, the adapter operands, the output
+    written (forward: X, W_nf4, sT, B, Y; backward: dY, W_nf4, sU, A, dX)."""
+    nb = c.N * c.K // 64
+    packed = c.N * c.K // 2 + nb + 4 * (-(-nb // 256)) + 4
+    return (2 * c.M * c.K + packed + 2 * c.M * c.r + 2 * c.r * c.N + 2 * c.M * c.N,
+            2 * c.M * c.N + packed + 2 * c.M * c.r + 2 * c.K * c.r + 2 * c.M * c.K)
 
 
 def fused_flops(c) -> tuple[float, float]:
@@ -503,7 +519,10 @@ def layer_record(name: str, ls: LayerSet, m: dict, world: int, steps: int, warmu
                      "frac_of_sustained": round(achieved / bf16_sus, 4) if bf16_sus else None,
                      "peak_source": f"{peak_src} bf16 burst",
                      "traffic": _traffic(TRAFFIC_CAPTURE, KERNEL_SOURCES, (name, dom)),
-                     "traffic_unit": f"bytes per step over the {nlin} {dom} launches (ncu dram read+write)"},
+                     "traffic_unit": f"bytes per step over the {nlin} {dom} launches (ncu dram read+write)"
+                                     + ("; scaled from the LLaMA-7B layer capture by algorithmic bytes"
+                                        if name in TRAFFIC_SCALED else ""),
+                     "algorithmic_bytes": sum(fused_bytes(c)[0 if dom == "fwd" else 1] for c in ls.cases)},
         "e2e": {"value": round(whole_job_rate(flops, world, m["e2e_ms_step"] * 1e-3) / 1e12, 3), "unit": "TFLOP/s",
                 "h2d_bytes_per_step": m["h2d"], "d2h_bytes_per_step": m["d2h"], "steps": m["e2e_steps"]},
         "gpu_launches": m["launches"],

@@ -46,3 +46,20 @@ def test_merge_bytes(api):
 def test_adamw_bytes_per_parameter():
     # read p, g, m, v (float32); write p, m, v (float32) and the bfloat16 copy
     assert bench.ADAMW_BYTES_PER_PARAM == 4 * 4 + 3 * 4 + 2
+
+
+def test_fused_gemm_bytes_and_scaled_traffic():
+    """The fused GEMMs' algorithmic bytes count the stored weight as the library
+    sizes it, and the 65B traffic figures are the LLaMA capture's traffic per
+    algorithmic byte applied to the 65B launches."""
+    for c in bench.layer_cases("proj7b"):
+        f, b = bench.fused_bytes(c)
+        packed = nf4.storage_bytes(c.N, c.K)
+        assert f == 2 * c.M * c.K + packed + 2 * c.M * c.r + 2 * c.r * c.N + 2 * c.M * c.N
+        assert b == 2 * c.M * c.N + packed + 2 * c.M * c.r + 2 * c.K * c.r + 2 * c.M * c.K
+    tc = bench.TRAFFIC_CAPTURE
+    for k, dom in ((0, "fwd"), (1, "bwd")):
+        llama = sum(bench.fused_bytes(c)[k] for c in bench.layer_cases("llama7b_layer"))
+        big = sum(bench.fused_bytes(c)[k] for c in bench.layer_cases("shapes_65b"))
+        want = big * tc[("llama7b_layer", dom)] / llama
+        assert abs(tc[("shapes_65b", dom)] - want) <= 1
