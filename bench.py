@@ -692,6 +692,92 @@ def measure_quantiser(n: int, k: int, steps: int, local: int, w_std: float = 0.0
             "bytes": "bf16 W read + stored weight written, per call (3 kernels), L2 flushed before each"}
 
 
+def run_quantiser(args):
+    """--workload quantiser: qlora_quantize alone on one weight (--n rows x --k
+    columns, default the 65B gate/up weight 22016 x 8192, N(0, 0.015) with 0.1%
+    outliers), L2 flushed before every call; GB/s of bf16 weight read plus stored
+    weight written."""
+    import torch
+    import torch.distributed as dist
+    from bit_nf4_quantised_codebook_b200 import api, inputs
+    world, rank, local = _dist()
+    _init_dist(world, local)
+    api.lib()
+    n, k = args.n, args.k
+    sampler = _gpu_sampler(local)
+    sampler.mark_start()
+    q = measure_quantiser(n, k, args.steps, local)
+    sampler.mark_end()
+    clocks = sampler.stop()
+    by = 2 * n * k + api.alloc_weight(n, k).nbytes()
+    dev = torch.device("cuda", local)
+    # end to end: the bf16 weight host -> device, quantise, the stored weight device -> host
+    W = api.bits_to_tensor(inputs.weight_bf16(n, k, 0.015, 0, 0.001), dev)
+    hw = W.cpu().pin_memory()
+    wq = api.alloc_weight(n, k, dev)
+    ws = torch.empty(api.qlora_workspace_size(api.QLORA_OP_QUANTIZE, 0, n, k, 0), dtype=torch.uint8, device=dev)
+    outs = [torch.empty_like(t, device="cpu").pin_memory() for t in (wq.codes, wq.c2q, wq.c1, wq.mean)]
+    e2e_steps = 5
+    torch.cuda.synchronize()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    launches0 = api.qlora_kernel_launch_count()
+    e0.record()
+    for _ in range(e2e_steps):
+        W.copy_(hw, non_blocking=True)
+        api.qlora_quantize(W, out=wq, ws=ws)
+        for h, d in zip(outs, (wq.codes, wq.c2q, wq.c1, wq.mean)):
+            h.copy_(d, non_blocking=True)
+    e1.record()
+    torch.cuda.synchronize()
+    e2e_ms = e0.elapsed_time(e1) / e2e_steps
+    launches = (api.qlora_kernel_launch_count() - launches0) // e2e_steps * args.steps
+    hbm, _, _, peak_src = _peaks()
+    line = {
+        "metric": "NF4 + double quantisation throughput (bf16 weight read, stored weight written)",
+        "value": round(whole_job_rate(by, world, q["ms"] * 1e-3) / 1e9, 2), "unit": "GB/s", "n_gpus": world,
+        "steps": args.steps, "warmup": 3, "ms_per_step": q["ms"], "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f32",
+        "data": "synthetic (seeded numpy N(0,0.015) with 0.1% 0.2*t(3) outliers, rounded to bf16)",
+        "config": {"workload": f"qlora_quantize on a {n}x{k} weight", "parallelism": f"replicas x{world}",
+                   "step": "one qlora_quantize call (block kernel, mean, E4M3 constants)",
+                   "l2": "a 256 MB buffer written before every call"},
+        "params_per_s": q["params_per_s"],
+        "roofline": {"kernel": "qlora_quantize (3 kernels)", "bound": "hbm", "achieved": q["gbs"], "peak": hbm,
+                     "unit": "GB/s", "frac": q["hbm_frac"], "peak_source": f"{peak_src} HBM copy", "traffic": None,
+                     "traffic_unit": "bytes per call (ncu dram read+write)"},
+        "e2e": {"value": round(by / (e2e_ms * 1e-3) / 1e9, 2), "unit": "GB/s", "h2d_bytes_per_step": 2 * n * k,
+                "d2h_bytes_per_step": wq.nbytes(), "steps": e2e_steps},
+        "gpu_launches": int(launches),
+        "clocks": clocks,
+    }
+    if world == 1 and rank == 0 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline_quantiser(n, k)
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+def cpu_baseline_quantiser(n: int, k: int, min_seconds: float = 10.0) -> dict:
+    """The oracle's quantiser on 256 rows of the weight, repeated; GB/s counted as on the GPU."""
+    from bit_nf4_quantised_codebook_b200 import inputs
+    from oracle import nf4
+    rows = 256
+    W = inputs.LinearCase("q", 1, rows, k, 8, 16.0, 0.015, 0.01, 0.01, 0.001, 0).W()
+    tot_t, reps = 0.0, 0
+    while tot_t < min_seconds or reps == 0:
+        t = time.perf_counter()
+        nf4.quantize_nf4(W)
+        tot_t += time.perf_counter() - t
+        reps += 1
+    by = reps * (2 * rows * k + nf4.storage_bytes(rows, k))
+    return {"value": round(by / tot_t / 1e9, 6), "unit": "GB/s", "cores": os.cpu_count(), "kind": "oracle",
+            "sample": f"{reps} x quantise {rows} rows x {k} drawn from the same recipe (float64/float32 numpy); "
+                      f"{tot_t:.1f} s"}
+
+
 # ---------------------------------------------------------------- the default line
 def run_ours(args):
     import torch
@@ -1359,9 +1445,10 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-sub", action="store_true", help="main line only (no sub-records)")
-    ap.add_argument("--workload", choices=list(WORKLOADS) + ["smallm", "adamw", "merge", "formats"],
+    ap.add_argument("--workload", choices=list(WORKLOADS) + ["smallm", "quantiser", "adamw", "merge", "formats"],
                     default="shapes_65b")
-    ap.add_argument("--n", type=int, default=8192, help="smallm: W rows (8192 or 28672)")
+    ap.add_argument("--n", type=int, default=None, help="smallm: W rows (8192 or 28672); quantiser: rows (22016)")
+    ap.add_argument("--k", type=int, default=8192, help="quantiser: columns")
     ap.add_argument("--m", type=int, default=16, help="smallm: tokens (1..64)")
     args = ap.parse_args()
     if args.impl == "ours":
@@ -1369,7 +1456,11 @@ def main():
     if args.impl == "reference":
         run_reference(args)
     elif args.workload == "smallm":
+        args.n = args.n or 8192
         run_smallm(args)
+    elif args.workload == "quantiser":
+        args.n = args.n or 22016
+        run_quantiser(args)
     elif args.workload == "adamw":
         run_adamw(args)
     elif args.workload == "merge":
