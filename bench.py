@@ -518,7 +518,8 @@ def layer_record(name: str, ls: LayerSet, m: dict, world: int, steps: int, warmu
                      "frac": round(achieved / bf16_burst, 4),
                      "frac_of_sustained": round(achieved / bf16_sus, 4) if bf16_sus else None,
                      "peak_source": f"{peak_src} bf16 burst",
-                     "traffic": _traffic(TRAFFIC_CAPTURE, KERNEL_SOURCES, (name, dom)),
+                     "traffic": (_traffic(TRAFFIC_CAPTURE, KERNEL_SOURCES, (name, dom))
+                                 if len(ls.cases) == len(layer_cases(name)) else None),
                      "traffic_unit": f"bytes per step over the {nlin} {dom} launches (ncu dram read+write)"
                                      + ("; scaled from the LLaMA-7B layer capture by algorithmic bytes"
                                         if name in TRAFFIC_SCALED else ""),
@@ -536,10 +537,16 @@ def layer_cases(name: str):
             "proj7b": lambda: [inputs.proj_7b()]}[name]()
 
 
-def measure_layer_set(name: str, steps: int, warmup: int, world: int, rank: int, local: int) -> dict:
+def measure_layer_set(name: str, steps: int, warmup: int, world: int, rank: int, local: int,
+                      only: str | None = None) -> dict:
     import torch
     dev = torch.device("cuda", local)
-    ls = LayerSet(layer_cases(name), dev, rank, world)
+    cases = layer_cases(name)
+    if only:  # one linear of the set (for a profiler capture of a single shape)
+        cases = [c for c in cases if c.name.split("_")[1] == only][:1]
+        if not cases:
+            raise SystemExit(f"--linear {only}: no such linear in {name}")
+    ls = LayerSet(cases, dev, rank, world)
     m = ls.measure(steps, warmup, world, local)
     rec = layer_record(name, ls, m, world, steps, warmup)
     del ls
@@ -788,10 +795,12 @@ def run_ours(args):
     _init_dist(world, local)
     api.lib()
     name = args.workload
-    line = measure_layer_set(name, args.steps, args.warmup, world, rank, local)
-    if name == "shapes_65b" and world == 1:
+    line = measure_layer_set(name, args.steps, args.warmup, world, rank, local, args.linear)
+    if args.linear:
+        line["config"]["linear"] = args.linear
+    if name == "shapes_65b" and world == 1 and not args.linear:
         line["quantiser"] = measure_quantiser(22016, 8192, 20, local)
-    if name == "shapes_65b" and world == 1 and not args.no_sub:
+    if name == "shapes_65b" and world == 1 and not args.no_sub and not args.linear:
         sub_steps = max(args.steps, 20)
         line["subrecords"] = {
             "proj7b": measure_layer_set("proj7b", max(args.steps, 50), max(args.warmup, 5), 1, 0, local),
@@ -799,7 +808,7 @@ def run_ours(args):
             "smallm": [measure_smallm(n, m, 500, 20, 1, local, e2e_steps=20)
                        for n in (8192, 28672) for m in (1, 16)],
         }
-    if world == 1 and rank == 0 and not args.no_cpu_baseline:
+    if world == 1 and rank == 0 and not args.no_cpu_baseline and not args.linear:
         line["cpu_baseline"] = cpu_baseline_layers(name)
     if rank == 0:
         print(json.dumps(line), flush=True)
@@ -1449,6 +1458,7 @@ def main():
                     default="shapes_65b")
     ap.add_argument("--n", type=int, default=None, help="smallm: W rows (8192 or 28672); quantiser: rows (22016)")
     ap.add_argument("--k", type=int, default=8192, help="quantiser: columns")
+    ap.add_argument("--linear", default=None, help="layer sets: run only this linear (q, k, v, o, gate, up, down)")
     ap.add_argument("--m", type=int, default=16, help="smallm: tokens (1..64)")
     args = ap.parse_args()
     if args.impl == "ours":
