@@ -74,18 +74,25 @@ def _peaks():
 # DRAM traffic (ncu dram__bytes_read.sum + dram__bytes_write.sum) of the dominant
 # kernels, from one-pass ncu launch-list captures, reported only while the kernel
 # sources hash to the build each capture was taken of (otherwise null).
-# Fused dequant GEMMs: `ncu --metrics gpu__time_duration.sum,dram__bytes_read.sum,
-# dram__bytes_write.sum --clock-control none -s 147 -c 42` over one step of the
-# LLaMA-7B layer set (`--workload llama7b_layer --steps 3 --warmup 3`); bytes per step
-# summed over the seven forward (fwd) or backward (bwd) launches.  The 65B set holds
-# about 5.5 GB on the device, more than a multi-metric capture should save and
-# restore, so its figures are the LLaMA capture's traffic per algorithmic byte
-# (0.842 fwd, 1.006 bwd) times the 65B launches' algorithmic bytes.
+# Fused dequant GEMMs, bytes per launch, keyed by (layer set, N, K, "fwd" | "bwd"):
+# `ncu --metrics gpu__time_duration.sum,dram__bytes_read.sum,dram__bytes_write.sum
+# --clock-control none -k regex:gemm_pair -s 6 -c 2` over `bench.py --linear <name>
+# --no-cpu-baseline --steps 3 --warmup 3` (one linear per step; the capture is the
+# first timed step's forward and backward launch), one run per weight shape of the
+# set (q, gate and down: k, v and o share q's shape, up shares gate's).  A set's
+# figure is the sum over its linears.
 KERNEL_SOURCES = ["gemm_pair.cuh", "gemm.cuh", "nf4_decode.cuh", "ptx.cuh", "launch.cuh", "linear.cu"]
-TRAFFIC_CAPTURE = {"sources_sha1": "b5144ea8dd10c7c950961b46652a80443e011c46",
-                   ("llama7b_layer", "fwd"): 634_221_568, ("llama7b_layer", "bwd"): 756_754_944,
-                   ("shapes_65b", "fwd"): 2_521_543_917, ("shapes_65b", "bwd"): 3_010_471_761}
-TRAFFIC_SCALED = {"shapes_65b"}
+TRAFFIC_CAPTURE = {"sources_sha1": "d1e611bffc63fb7fa183aa54d0ae0d3bc560c901",
+                   ("shapes_65b", 8192, 8192, "fwd"): 526_467_840, ("shapes_65b", 8192, 8192, "bwd"): 497_913_856,
+                   ("shapes_65b", 22016, 8192, "fwd"): 1_031_215_872,
+                   ("shapes_65b", 22016, 8192, "bwd"): 1_419_983_360,
+                   ("shapes_65b", 8192, 22016, "fwd"): 1_412_864_512,
+                   ("shapes_65b", 8192, 22016, "bwd"): 1_060_189_696,
+                   ("llama7b_layer", 4096, 4096, "fwd"): 46_133_248, ("llama7b_layer", 4096, 4096, "bwd"): 44_052_736,
+                   ("llama7b_layer", 11008, 4096, "fwd"): 118_332_928,
+                   ("llama7b_layer", 11008, 4096, "bwd"): 194_748_928,
+                   ("llama7b_layer", 4096, 11008, "fwd"): 198_091_008,
+                   ("llama7b_layer", 4096, 11008, "bwd"): 114_373_888}
 # The small-M kernel: the same one-pass capture of `--workload smallm`, bytes per launch, per (N, M).
 SMALLM_SOURCES = ["gemm_smallm.cuh", "gemm.cuh", "nf4_decode.cuh", "ptx.cuh", "launch.cuh", "linear.cu"]
 SMALLM_TRAFFIC = {"sources_sha1": None}
@@ -107,6 +114,15 @@ def _traffic(table, files, key):
     if table.get("sources_sha1") and table["sources_sha1"] == kernel_sources_sha1(files):
         return table.get(key)
     return None
+
+
+def fused_traffic(name: str, cases, dom: str, table=None, files=None):
+    """DRAM bytes of the fused GEMM launches (forward or backward) of `cases`:
+    the sum of the per-shape captures, or None if any shape is missing or the
+    kernel sources have changed since the capture."""
+    table = TRAFFIC_CAPTURE if table is None else table
+    vals = [_traffic(table, files or KERNEL_SOURCES, (name, c.N, c.K, dom)) for c in cases]
+    return None if not vals or any(v is None for v in vals) else int(sum(vals))
 
 
 class ClockSampler:
@@ -518,11 +534,9 @@ def layer_record(name: str, ls: LayerSet, m: dict, world: int, steps: int, warmu
                      "frac": round(achieved / bf16_burst, 4),
                      "frac_of_sustained": round(achieved / bf16_sus, 4) if bf16_sus else None,
                      "peak_source": f"{peak_src} bf16 burst",
-                     "traffic": (_traffic(TRAFFIC_CAPTURE, KERNEL_SOURCES, (name, dom))
-                                 if len(ls.cases) == len(layer_cases(name)) else None),
-                     "traffic_unit": f"bytes per step over the {nlin} {dom} launches (ncu dram read+write)"
-                                     + ("; scaled from the LLaMA-7B layer capture by algorithmic bytes"
-                                        if name in TRAFFIC_SCALED else ""),
+                     "traffic": fused_traffic(name, ls.cases, dom),
+                     "traffic_unit": f"bytes per step over the {nlin} {dom} launches (ncu dram read+write, "
+                                     f"one capture per weight shape)",
                      "algorithmic_bytes": sum(fused_bytes(c)[0 if dom == "fwd" else 1] for c in ls.cases)},
         "e2e": {"value": round(whole_job_rate(flops, world, m["e2e_ms_step"] * 1e-3) / 1e12, 3), "unit": "TFLOP/s",
                 "h2d_bytes_per_step": m["h2d"], "d2h_bytes_per_step": m["d2h"], "steps": m["e2e_steps"]},

@@ -69,6 +69,11 @@ struct GemmParams {
   int cluster;       // K splits = CTAs per cluster along z (1, 2, 4 or 8)
   int red_cols;      // valid output columns (<= BN)
   float scale;       // applied to the reduced sum
+  // CTA-pair kernel only: tile order.  0 = the launch grid's order (token tiles
+  // fastest); g > 0 = groups of g token-pair tiles, all W-side tiles of a group
+  // before the next group, so that the activation tiles the resident CTAs share
+  // stay in L2 while the W tiles stream past them.
+  int raster_gm;
 };
 
 template <int BN_, int STAGES_, bool A_MN_, int BMODE_, int LORA_, int OUT_>

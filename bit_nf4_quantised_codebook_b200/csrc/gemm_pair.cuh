@@ -93,8 +93,20 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(C::NUM_THREADS, 1)
   const int lane = threadIdx.x & 31;
   const uint32_t rank = cluster_ctarank();
   const bool leader = rank == 0;
-  const int m0 = blockIdx.x * 128 * C::MSUB;  // this CTA's token rows (MSUB sub-tiles of 128)
-  const int n0 = blockIdx.y * C::BN;          // the pair's W-side tile
+  // the pair's tile (tm: token-pair tile, tn: W-side tile); both CTAs of a pair
+  // compute the same indices from the pair's position in the launch order
+  int tm = static_cast<int>(blockIdx.x >> 1), tn = static_cast<int>(blockIdx.y);
+  if (p.raster_gm > 0) {
+    const int tmp = static_cast<int>(gridDim.x >> 1), tnn = static_cast<int>(gridDim.y);
+    const int pidx = tn * tmp + tm;                      // launch order: x fastest
+    const int group = pidx / (p.raster_gm * tnn);
+    const int within = pidx - group * p.raster_gm * tnn;
+    const int rows = tmp - group * p.raster_gm < p.raster_gm ? tmp - group * p.raster_gm : p.raster_gm;
+    tm = group * p.raster_gm + within % rows;
+    tn = within / rows;
+  }
+  const int m0 = (2 * tm + static_cast<int>(rank)) * 128 * C::MSUB;  // this CTA's token rows
+  const int n0 = tn * C::BN;                                          // the pair's W-side tile
   const int nh0 = n0 + 128 * static_cast<int>(rank);  // this CTA's half of it
   const int split = blockIdx.z;
   const int kb_begin = split * p.k_iters;

@@ -164,6 +164,19 @@ static cudaError_t run_skinny(SkinnyKind kind, const LaunchCtx &c, const SplitPl
 }
 
 // ---------------------------------------------------------------- fused dequant GEMM
+#ifndef QLORA_RASTER_GROUP
+#define QLORA_RASTER_GROUP 4
+#endif
+// Token-pair tiles per raster group of the CTA-pair kernel (0: the launch
+// grid's order).  The 74 CTA pairs resident at a time then cover about 4 token
+// tiles x 18 W tiles: a wave reads 4 activation tiles (1 KiB per reduction
+// index each) and 18 W tiles (about 133 bytes per reduction index each) from
+// DRAM, close to the minimum of 1024·a + 133·b over a·b = 74 (a ≈ 3); the
+// grid's own order (all 16 token tiles of M = 8192 with 4-5 W tiles) reads
+// about 2.6 times as much.  Consecutive waves of a group share its activation
+// tiles, which L2 keeps when they fit.
+constexpr int kRasterGroup = QLORA_RASTER_GROUP;
+
 // fwd: D[M x N] = X·W_hatᵀ + sT·B       (W-side operand K-major: rows of W)
 // bwd: D[M x K] = dY·W_hat + sU·Aᵀ      (W-side operand MN-major: columns of W)
 // `pair` selects the CTA-pair kernel (256-token tiles); otherwise one CTA per
@@ -202,6 +215,10 @@ static cudaError_t run_fused(bool fwd, const LaunchCtx &c, const qlora_nf4_weigh
   p.split_stride = M * n_out;
   const unsigned gx = pair ? static_cast<unsigned>(2 * ((M + kPairTokens - 1) / kPairTokens))
                            : static_cast<unsigned>((M + 127) / 128);
+  if (pair && kRasterGroup > 0) {
+    const int tmp = static_cast<int>(gx / 2);
+    p.raster_gm = kRasterGroup < tmp ? kRasterGroup : tmp;
+  }
   dim3 grid(gx, static_cast<unsigned>((n_out + 255) / 256), static_cast<unsigned>(sp.splits));
   if (ev0) cudaEventRecord(ev0, c.stream);
   if (pair) {

@@ -48,18 +48,30 @@ def test_adamw_bytes_per_parameter():
     assert bench.ADAMW_BYTES_PER_PARAM == 4 * 4 + 3 * 4 + 2
 
 
-def test_fused_gemm_bytes_and_scaled_traffic():
+def test_fused_gemm_bytes_and_per_shape_traffic():
     """The fused GEMMs' algorithmic bytes count the stored weight as the library
-    sizes it, and the 65B traffic figures are the LLaMA capture's traffic per
-    algorithmic byte applied to the 65B launches."""
+    sizes it, and a layer set's DRAM traffic is the sum of its linears'
+    per-shape captures (q, k, v, o share one shape, gate and up another), or
+    None once a shape is missing or the kernel sources differ from the capture's."""
     for c in bench.layer_cases("proj7b"):
         f, b = bench.fused_bytes(c)
         packed = nf4.storage_bytes(c.N, c.K)
         assert f == 2 * c.M * c.K + packed + 2 * c.M * c.r + 2 * c.r * c.N + 2 * c.M * c.N
         assert b == 2 * c.M * c.N + packed + 2 * c.M * c.r + 2 * c.K * c.r + 2 * c.M * c.K
-    tc = bench.TRAFFIC_CAPTURE
-    for k, dom in ((0, "fwd"), (1, "bwd")):
-        llama = sum(bench.fused_bytes(c)[k] for c in bench.layer_cases("llama7b_layer"))
-        big = sum(bench.fused_bytes(c)[k] for c in bench.layer_cases("shapes_65b"))
-        want = big * tc[("llama7b_layer", dom)] / llama
-        assert abs(tc[("shapes_65b", dom)] - want) <= 1
+    cases = bench.layer_cases("shapes_65b")
+    shapes = {(c.N, c.K) for c in cases}
+    assert shapes == {(8192, 8192), (22016, 8192), (8192, 22016)}
+    sha = bench.kernel_sources_sha1()
+    table = {"sources_sha1": sha}
+    for n, (N, K) in enumerate(sorted(shapes)):
+        table[("shapes_65b", N, K, "fwd")] = 1000 * (n + 1)
+        table[("shapes_65b", N, K, "bwd")] = 7 * (n + 1)
+    # sorted shapes: (8192, 8192) x4 -> 1, (8192, 22016) x1 -> 2, (22016, 8192) x2 -> 3
+    assert bench.fused_traffic("shapes_65b", cases, "fwd", table) == 1000 * (4 * 1 + 1 * 2 + 2 * 3)
+    assert bench.fused_traffic("shapes_65b", cases, "bwd", table) == 7 * (4 * 1 + 1 * 2 + 2 * 3)
+    one = [c for c in cases if c.name.split("_")[1] == "gate"]
+    assert bench.fused_traffic("shapes_65b", one, "fwd", table) == 3000
+    del table[("shapes_65b", 8192, 22016, "bwd")]
+    assert bench.fused_traffic("shapes_65b", cases, "bwd", table) is None
+    table["sources_sha1"] = "0" * 40
+    assert bench.fused_traffic("shapes_65b", cases, "fwd", table) is None
