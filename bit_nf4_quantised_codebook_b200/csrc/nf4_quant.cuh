@@ -32,7 +32,7 @@ constexpr int kBuckets = 64;
 constexpr float kBucketScale = 32.0f;          // buckets per unit of x_hat
 constexpr float kBucketMargin = 1.0f / 1024;   // widening on each side
 
-struct CodeBucket {
+struct __align__(8) CodeBucket {  // 8-byte aligned: one 64-bit shared-memory load per lookup
   int base;
   float thr;
 };

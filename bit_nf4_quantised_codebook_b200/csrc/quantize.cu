@@ -155,25 +155,28 @@ __global__ void __launch_bounds__(kQThreads, 1) k_quant_blocks(const uint16_t *_
         x[2 * i] = __uint_as_float(u[i] << 16);
         x[2 * i + 1] = __uint_as_float(u[i] & 0xFFFF0000u);
       }
-      float amax = 0.f;
+      // absmax on the bit patterns: with the sign cleared, bfloat16 magnitudes
+      // order like unsigned integers, two per 16x2 max; a block maximum at or
+      // above 0x7F80 (the infinity pattern) means an infinity or NaN in the block
+      uint32_t m2 = 0;
 #pragma unroll
-      for (int i = 0; i < 8; ++i) {
-        const float av = fabsf(x[i]);
-        bad |= !(av <= 3.402823466e38f);
-        amax = fmaxf(amax, av);
-      }
-      amax = fmaxf(amax, __shfl_xor_sync(0xFFFFFFFFu, amax, 1));
-      amax = fmaxf(amax, __shfl_xor_sync(0xFFFFFFFFu, amax, 2));
-      amax = fmaxf(amax, __shfl_xor_sync(0xFFFFFFFFu, amax, 4));
+      for (int i = 0; i < 4; ++i) m2 = __vmaxu2(m2, u[i] & 0x7FFF7FFFu);
+      uint32_t mb = max(m2 & 0xFFFFu, m2 >> 16);
+      mb = max(mb, __shfl_xor_sync(0xFFFFFFFFu, mb, 1));
+      mb = max(mb, __shfl_xor_sync(0xFFFFFFFFu, mb, 2));
+      mb = max(mb, __shfl_xor_sync(0xFFFFFFFFu, mb, 4));
+      const float amax = __uint_as_float(mb << 16);
       uint32_t packed = 0x77777777u;  // all-zero block: every code is the zero level
-      if (amax >= kFastQuotientMinAbsmax) {
+      if (mb >= 0x7F80u) {
+        bad = true;  // reported; the block keeps the zero-level codes (the bucket index needs |x_hat| <= 1)
+      } else if (amax >= kFastQuotientMinAbsmax) {
         const float ra = __frcp_rn(amax);
         packed = 0;
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
           const uint32_t hi = lane_centred_code(quotient_rn(x[2 * i], amax, ra), tab, lane);
           const uint32_t lo = lane_centred_code(quotient_rn(x[2 * i + 1], amax, ra), tab, lane);
-          packed |= ((hi << 4) | lo) << (8 * i);
+          packed += (lo + (hi << 4)) << (8 * i);  // disjoint nibbles: + is |
         }
       } else if (amax > 0.f) {
         packed = 0;
@@ -181,7 +184,7 @@ __global__ void __launch_bounds__(kQThreads, 1) k_quant_blocks(const uint16_t *_
         for (int i = 0; i < 4; ++i) {
           const uint32_t hi = nf4_code(__fdiv_rn(x[2 * i], amax), thr);
           const uint32_t lo = nf4_code(__fdiv_rn(x[2 * i + 1], amax), thr);
-          packed |= ((hi << 4) | lo) << (8 * i);
+          packed += (lo + (hi << 4)) << (8 * i);
         }
       }
       if (valid) {
