@@ -28,9 +28,13 @@
 // rank 0's producer waits on the predecessor, right before loading sT, and the
 // main loop overlaps the predecessor's tail.
 //
-// Roles (320 threads, 2 CTAs per SM): warp 0 TMA producer, warp 1 TMEM
-// allocator and MMA issuer, warps 2..9 two dequant groups of 4 warps (one warp
-// per TMEM lane quadrant) taking alternate K steps.  The E4M3 block constants
+// Roles (352 threads, 2 CTAs per SM): warp 0 TMA producer, warp 1 TMEM
+// allocator and MMA issuer of dequant group 0, warps 2..9 two dequant groups of
+// 4 warps (one warp per TMEM lane quadrant) taking alternate K steps, warp 10
+// the MMA issuer of group 1.  Each issuer accumulates its group's steps in its
+// own TMEM accumulator (two MMA streams per CTA; a single issuing thread paces
+// the MMAs of 128 x NT x 16 well below the tensor pipe's rate), and the two are
+// added when the partial is parked.  The E4M3 block constants
 // and fp32 group scales of the CTA's weight slice are staged in shared memory
 // once, by the dequant threads, with coalesced loads.
 #pragma once
@@ -53,7 +57,11 @@ struct SmallCfg {
   static constexpr int C_ROW = 32 * KB;          // bytes of packed codes per W row and step
   static constexpr int C_BYTES = 128 * C_ROW;    // swizzled with the C_ROW-byte TMA swizzle
   static constexpr int STAGE_BYTES = KB * X_BYTES + C_BYTES;
-  static constexpr int TSLOTS = 6 / KB;          // TMEM A slots (KB x 32 columns each), 192 columns in all
+  static constexpr int ACC_COLS = NT < 32 ? 32 : NT;
+  static constexpr int TMEM_COLS = 256;
+  static constexpr int NACC = 2;                 // one accumulator per dequant group and its MMA issuer
+  static constexpr int TSLOTS_FIT = (TMEM_COLS - NACC * ACC_COLS) / (32 * KB);
+  static constexpr int TSLOTS = TSLOTS_FIT < 6 / KB ? TSLOTS_FIT : 6 / KB;  // TMEM A slots (KB x 32 columns each)
   // Shared-memory ring: an even number of stages, so that with two dequant groups taking
   // alternate steps every stage belongs to one group, and each full-barrier phase is
   // awaited in order by a single consumer (a parity wait only tells apart the phase it
@@ -69,14 +77,14 @@ struct SmallCfg {
   static constexpr int OFF_C1 = OFF_Q8 + 128 * Q8_STRIDE_MAX;
   static constexpr int OFF_BAR = (OFF_C1 + kSmallC1Max * 4 + 7) & ~7;
   static constexpr int SMEM_BYTES = OFF_BAR + 256 + 1024;  // + alignment slack
-  static constexpr int ACC_COLS = NT < 32 ? 32 : NT;
-  static constexpr int TMEM_COLS = 256;
   static constexpr int PSTRIDE = 128 + 4;  // floats per token row of the parked partial
   static constexpr int P_BYTES = NT * PSTRIDE * 4;
   static constexpr int DQ_THREADS = 128 * GROUPS;
-  static constexpr int NUM_THREADS = 64 + DQ_THREADS;
+  static constexpr int ISSUER1_WARP = 2 + 4 * GROUPS;  // the second MMA issuer, after the dequant warps
+  static constexpr int NUM_THREADS = 64 + DQ_THREADS + 32;
   static_assert(NT % 16 == 0 && NT >= 16 && NT <= 64, "token tile");
-  static_assert(ACC_COLS + TSLOTS * 32 * KB <= TMEM_COLS, "TMEM budget");
+  static_assert(NACC * ACC_COLS + TSLOTS * 32 * KB <= TMEM_COLS, "TMEM budget");
+  static_assert(GROUPS == NACC, "each dequant group has its own issuer and accumulator");
   static_assert(STAGES >= TSLOTS, "a slot's barrier phase is never overtaken before its waiter checks it");
   static_assert(STAGE_BYTES % 1024 == 0 && X_BYTES % 1024 == 0, "swizzle atoms stay 1024-byte aligned");
   static_assert(P_BYTES <= RING_BYTES, "the partial is parked in the drained ring");
@@ -145,7 +153,7 @@ __global__ void __launch_bounds__(C::NUM_THREADS, 2)
     }
     mbar_init(lfull, 1);
     mbar_init(lempty, 1);
-    mbar_init(acc_full, 1);
+    mbar_init(acc_full, C::NACC);  // one commit per issuer
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -205,9 +213,14 @@ __global__ void __launch_bounds__(C::NUM_THREADS, 2)
         mbar_wait_bounded(lfull, (lissued - 1) & 1, &dummy, nullptr, kDrainNs);
       }
     }
-  } else if (warp == 1) {
-    // ------------------------------------------------------------ MMA issuer
+  } else if (warp == 1 || warp == C::ISSUER1_WARP) {
+    // ------------------------------------------------------------ MMA issuers
+    // Issuer g (warp 1: g = 0, the last warp: g = 1) takes the steps of dequant group g
+    // (j = g, g + 2, ...) into its own accumulator, so two MMA streams per CTA are in
+    // flight; issuer 0 then adds the adapter product to its accumulator.
     if (lane == 0) {
+      const int g = warp == 1 ? 0 : 1;
+      const uint32_t acc_t = tmem_base + g * C::ACC_COLS;
       constexpr uint32_t idesc_main = idesc_bf16(128, C::NT, false, false);
       constexpr uint32_t idesc_lora = idesc_bf16(128, C::NT, true, false);
       bool ok = true;
@@ -215,35 +228,30 @@ __global__ void __launch_bounds__(C::NUM_THREADS, 2)
       // +X_BYTES >> 4 per block, +STAGE_BYTES >> 4 per ring stage
       const uint64_t desc0 = smem_desc_sw128(smem_base, 16, 1024);
       uint32_t acc = 0;  // the first MMA overwrites the accumulator
-      int s = 0;
-      uint32_t ph = 0;
-      for (int j = 0; j < n_ss; ++j) {
-        if (!mbar_wait_bounded(&ready[s], ph, abort_flag, p.dev_err, p.timeout_ns)) {
+      for (int j = g; j < n_ss; j += C::NACC) {
+        const int s = j % C::STAGES;
+        if (!mbar_wait_bounded(&ready[s], (j / C::STAGES) & 1, abort_flag, p.dev_err, p.timeout_ns)) {
           ok = false;
           break;
         }
         tc_fence_after();
         const uint64_t bd = desc0 + static_cast<uint64_t>((s * C::STAGE_BYTES) >> 4);
-        const uint32_t a_tmem = tmem_base + C::ACC_COLS + (j % C::TSLOTS) * 32 * C::KB;
+        const uint32_t a_tmem = tmem_base + C::NACC * C::ACC_COLS + (j % C::TSLOTS) * 32 * C::KB;
         const bool two = n_main - j * C::KB >= 2;
 #pragma unroll
         for (int kk = 0; kk < 4; ++kk) {
-          mma_bf16_ts(tmem_base, a_tmem + kk * 8, bd + 2 * kk, idesc_main, acc);
+          mma_bf16_ts(acc_t, a_tmem + kk * 8, bd + 2 * kk, idesc_main, acc);
           acc = 1;
         }
         if (C::KB == 2 && two) {
 #pragma unroll
           for (int kk = 0; kk < 4; ++kk)
-            mma_bf16_ts(tmem_base, a_tmem + 32 + kk * 8, bd + (C::X_BYTES >> 4) + 2 * kk, idesc_main, 1u);
+            mma_bf16_ts(acc_t, a_tmem + 32 + kk * 8, bd + (C::X_BYTES >> 4) + 2 * kk, idesc_main, 1u);
         }
         mma_commit(&empty[s]);
-        if (++s == C::STAGES) {
-          s = 0;
-          ph ^= 1;
-        }
       }
       bool first = acc == 0;
-      for (int c = 0; ok && c < n_lora; ++c) {
+      for (int c = 0; g == 0 && ok && c < n_lora; ++c) {
         if (!mbar_wait_bounded(lfull, c & 1, abort_flag, p.dev_err, p.timeout_ns)) break;
         tc_fence_after();
         const int rem = p.lora_r - c * 64;
@@ -251,13 +259,13 @@ __global__ void __launch_bounds__(C::NUM_THREADS, 2)
         const uint32_t a_base = smem_base + C::OFF_LA;
         const uint32_t b_base = smem_base + C::OFF_LX;
         for (int kk = 0; kk < ksteps; ++kk) {
-          mma_bf16_ss(tmem_base, smem_desc_sw128(a_base + kk * 2048, 8192, 1024),
+          mma_bf16_ss(acc_t, smem_desc_sw128(a_base + kk * 2048, 8192, 1024),
                       smem_desc_sw128(b_base + kk * 32, 16, 1024), idesc_lora, first ? 0u : 1u);
           first = false;
         }
         mma_commit(lempty);
       }
-      mma_commit(acc_full);  // tracks completion of everything issued above
+      mma_commit(acc_full);  // tracks completion of everything this issuer issued
     }
   } else {
     // ------------------------------------------------------------ dequant groups (warps 2..9)
@@ -330,7 +338,7 @@ __global__ void __launch_bounds__(C::NUM_THREADS, 2)
     // the 8 lanes of one shared-memory phase (rows i..i+7) cover all 32 banks
     const uint32_t sw = C::KB == 2 ? (row >> 1) & 3 : (row >> 2) & 1;
     const uint32_t c_row = smem_base + C::KB * C::X_BYTES + row * C::C_ROW;
-    const uint32_t t_row = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + C::ACC_COLS;
+    const uint32_t t_row = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + C::NACC * C::ACC_COLS;
     // block index of (row, block i) relative to the first staged group scale
     const int rb = static_cast<int>(static_cast<int64_t>(n0 + row) * kbt + kb_begin - (gfirst << 8));
     const uint8_t *q8row = q8s + row * qs;
@@ -383,15 +391,24 @@ __global__ void __launch_bounds__(C::NUM_THREADS, 2)
       if (__all_sync(0xFFFFFFFFu, got) && !*abort_flag) {
         tc_fence_after();
         float *P = reinterpret_cast<float *>(smem);
-        const bool any = n_main > 0 || lora;
+        // accumulator 0 holds steps 0, 2, ... and the adapter product; accumulator 1 steps 1, 3, ...
+        const bool w0 = n_ss >= 1 || n_lora > 0, w1 = n_ss >= 2;
+        const uint32_t lane_base = tmem_base + (static_cast<uint32_t>(q * 32) << 16);
 #pragma unroll
         for (int c0 = 0; c0 < C::NT; c0 += 32) {
           uint32_t v[32];
-          tmem_ld32(tmem_base + (static_cast<uint32_t>(q * 32) << 16) + c0, v);
+          tmem_ld32(lane_base + c0, v);
           tmem_ld_wait();
 #pragma unroll
           for (int j = 0; j < 32; ++j)
-            if (c0 + j < C::NT) P[(c0 + j) * C::PSTRIDE + row] = any ? __uint_as_float(v[j]) : 0.f;
+            if (c0 + j < C::NT) P[(c0 + j) * C::PSTRIDE + row] = w0 ? __uint_as_float(v[j]) : 0.f;
+          if (w1) {
+            tmem_ld32(lane_base + C::ACC_COLS + c0, v);
+            tmem_ld_wait();
+#pragma unroll
+            for (int j = 0; j < 32; ++j)
+              if (c0 + j < C::NT) P[(c0 + j) * C::PSTRIDE + row] += __uint_as_float(v[j]);
+          }
         }
       }
     }
