@@ -46,7 +46,11 @@
 
 namespace qlora {
 
-constexpr int kSmallC1Max = 260;     // group scales a CTA can touch: (127·512 + 64)/256 + 2, rounded up
+constexpr int kSmallC1Max = 260;
+// Pipeline waits sleep in the barrier (up to this long per poll) instead of
+// spinning, so waiting warps leave the issue slots and the integer pipe to the
+// decoding ones.
+constexpr uint32_t kSmallWaitHintNs = 1000;     // group scales a CTA can touch: (127·512 + 64)/256 + 2, rounded up
 
 template <int NT_, int GROUPS_>
 struct SmallCfg {
@@ -182,7 +186,7 @@ __global__ void __launch_bounds__(C::NUM_THREADS, 2)
       for (int j = 0; j < n_ss; ++j) {
         const int s = j % C::STAGES;
         const uint32_t ph = (j / C::STAGES) & 1;
-        if (!mbar_wait_bounded(&empty[s], ph ^ 1, abort_flag, p.dev_err, p.timeout_ns)) break;
+        if (!mbar_wait_bounded_sleep(&empty[s], ph ^ 1, abort_flag, p.dev_err, p.timeout_ns, kSmallWaitHintNs)) break;
         uint8_t *st = smem + s * C::STAGE_BYTES;
         const int kb = kb_begin + j * C::KB;
         mbar_arrive_expect_tx(&full[s], C::STAGE_BYTES);
@@ -230,7 +234,8 @@ __global__ void __launch_bounds__(C::NUM_THREADS, 2)
       uint32_t acc = 0;  // the first MMA overwrites the accumulator
       for (int j = g; j < n_ss; j += C::NACC) {
         const int s = j % C::STAGES;
-        if (!mbar_wait_bounded(&ready[s], (j / C::STAGES) & 1, abort_flag, p.dev_err, p.timeout_ns)) {
+        if (!mbar_wait_bounded_sleep(&ready[s], (j / C::STAGES) & 1, abort_flag, p.dev_err, p.timeout_ns,
+                                     kSmallWaitHintNs)) {
           ok = false;
           break;
         }
@@ -347,13 +352,14 @@ __global__ void __launch_bounds__(C::NUM_THREADS, 2)
       const uint32_t ph = (j / C::STAGES) & 1;
       const uint32_t slot = t_row + (j % C::TSLOTS) * 32 * C::KB;
       const int nb = n_main - j * C::KB < C::KB ? n_main - j * C::KB : C::KB;
-      const bool okf = mbar_wait_bounded(&full[s], ph, abort_flag, p.dev_err, p.timeout_ns);
+      const bool okf = mbar_wait_bounded_sleep(&full[s], ph, abort_flag, p.dev_err, p.timeout_ns, kSmallWaitHintNs);
       if (!__all_sync(0xFFFFFFFFu, okf)) break;
       if (j >= C::TSLOTS) {
         // the MMAs that last read this TMEM slot (step j - TSLOTS) are complete
         const int jp = j - C::TSLOTS;
         const bool oke =
-            mbar_wait_bounded(&empty[jp % C::STAGES], (jp / C::STAGES) & 1, abort_flag, p.dev_err, p.timeout_ns);
+            mbar_wait_bounded_sleep(&empty[jp % C::STAGES], (jp / C::STAGES) & 1, abort_flag, p.dev_err, p.timeout_ns,
+                                    kSmallWaitHintNs);
         if (!__all_sync(0xFFFFFFFFu, oke)) break;
       }
       tc_fence_after();

@@ -50,6 +50,20 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, uint32_t parity) {
   return ok != 0;
 }
 
+// try_wait with a suspend-time hint: the thread may sleep up to `hint_ns` for the
+// phase instead of returning at once, so waiting warps spend no issue slots.
+__device__ __forceinline__ bool mbar_try_wait_hint(uint64_t *bar, uint32_t parity, uint32_t hint_ns) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.acquire.cta.shared::cta.b64 p, [%1], %2, %3;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity), "r"(hint_ns)
+      : "memory");
+  return ok != 0;
+}
+
 // Bounded wait.  Returns false when the wait gave up: either *abort was raised
 // by another role of the CTA or `timeout_ns` elapsed (then *abort is raised and
 // QLORA_DEVERR_TIMEOUT is OR-ed into *dev_err).
@@ -60,6 +74,25 @@ __device__ __forceinline__ bool mbar_wait_bounded(uint64_t *bar, uint32_t parity
   for (uint32_t it = 1;; ++it) {
     if (mbar_try_wait(bar, parity)) return true;
     if ((it & 63) == 0) {
+      if (*abort) return false;
+      if (globaltimer_ns() - t0 > timeout_ns) {
+        *abort = 1;
+        if (dev_err) atomicOr(dev_err, 2);
+        return false;
+      }
+    }
+  }
+}
+
+// The same bounded wait with sleeping polls (mbar_try_wait_hint); *abort and the
+// clock are checked every 8 polls.
+__device__ __forceinline__ bool mbar_wait_bounded_sleep(uint64_t *bar, uint32_t parity, volatile int *abort,
+                                                        int *dev_err, uint64_t timeout_ns, uint32_t hint_ns) {
+  if (mbar_try_wait(bar, parity)) return true;
+  uint64_t t0 = globaltimer_ns();
+  for (uint32_t it = 1;; ++it) {
+    if (mbar_try_wait_hint(bar, parity, hint_ns)) return true;
+    if ((it & 7) == 0) {
       if (*abort) return false;
       if (globaltimer_ns() - t0 > timeout_ns) {
         *abort = 1;
