@@ -399,6 +399,107 @@ class LayerSet:
         if ev is not None:
             api.qlora_set_timing_events()
 
+    def e2e(self, e2e_steps: int, world: int) -> tuple[float, int, int]:
+        """Device time of `e2e_steps` training steps with every input copied in from
+        pinned host memory and every output copied back, the copies on their own
+        streams so that they overlap the compute and each other (host-to-device and
+        device-to-host run on separate copy engines).  X, dY, Y and dX are double
+        buffered by step parity; event waits keep every buffer from being refilled
+        before its last reader is done.  Returns (ms, h2d bytes, d2h bytes) per step."""
+        import torch
+        nl = len(self.lin)
+        h_in = [{k: torch.empty_like(L[k], device="cpu").pin_memory() for k in ("X", "dY")} for L in self.lin]
+        for h, L in zip(h_in, self.lin):
+            for k in h:
+                h[k].copy_(L[k])
+        h_out = [{k: torch.empty_like(L[k], device="cpu").pin_memory() for k in ("Y", "dX")} for L in self.lin]
+        h_grad = torch.empty_like(self.bucket, device="cpu").pin_memory()
+        h2d = sum(t.numel() * t.element_size() for h in h_in for t in h.values())
+        d2h = sum(t.numel() * t.element_size() for h in h_out for t in h.values()) + h_grad.numel() * 4
+        bufs = [[{k: L[k] for k in ("X", "dY", "Y", "dX")} for L in self.lin],
+                [{k: torch.empty_like(L[k]) for k in ("X", "dY", "Y", "dX")} for L in self.lin]]
+        main = torch.cuda.current_stream()
+        s_in, s_out = torch.cuda.Stream(), torch.cuda.Stream()
+
+        def events():
+            return [torch.cuda.Event() for _ in range(nl)]
+
+        # per parity: inputs landed, forward done, backward done, outputs copied out
+        in_x, in_dy, fwd_done, bwd_done, out_y, out_dx = ([events(), events()] for _ in range(6))
+        grad_out = torch.cuda.Event()
+        api = self.api
+        if world > 1:
+            import torch.distributed as dist
+            dist.barrier()
+        torch.cuda.synchronize()
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        e0.record(main)
+        s_in.wait_event(e0)
+        s_out.wait_event(e0)
+        for st in range(e2e_steps):
+            p, old = st % 2, st >= 2  # `old`: the buffers of parity p were used two steps ago
+            B = bufs[p]
+            with torch.cuda.stream(s_in):
+                for i in range(nl):
+                    if old:
+                        s_in.wait_event(bwd_done[p][i])  # the last reader of X_i and dY_i
+                    B[i]["X"].copy_(h_in[i]["X"], non_blocking=True)
+                    in_x[p][i].record(s_in)
+                for i in reversed(range(nl)):
+                    B[i]["dY"].copy_(h_in[i]["dY"], non_blocking=True)
+                    in_dy[p][i].record(s_in)
+            for i, L in enumerate(self.lin):
+                main.wait_event(in_x[p][i])
+                if old:
+                    main.wait_event(out_y[p][i])  # Y_i of two steps ago has been copied out
+                api.qlora_linear_forward(L["q"], B[i]["X"], L["A"], L["B"], L["case"].s, Y=B[i]["Y"],
+                                         T_save=L["sT"], ws=self.ws_f, dev_err=self.err)
+                fwd_done[p][i].record(main)
+            if st >= 1:
+                main.wait_event(grad_out)  # the previous step's gradients have been copied out
+            for i in reversed(range(nl)):
+                L = self.lin[i]
+                main.wait_event(in_dy[p][i])
+                if old:
+                    main.wait_event(out_dx[p][i])
+                api.qlora_linear_backward(L["q"], B[i]["X"], B[i]["dY"], L["A"], L["B"], L["case"].s,
+                                          T_saved=L["sT"], dX=B[i]["dX"], dA=L["dA"], dB=L["dB"], ws=self.ws_b,
+                                          dev_err=self.err)
+                bwd_done[p][i].record(main)
+            if world > 1:
+                allreduce_grads(self.bucket)
+            grads_ready = torch.cuda.Event()
+            grads_ready.record(main)
+            with torch.cuda.stream(s_out):
+                for i in range(nl):
+                    s_out.wait_event(fwd_done[p][i])
+                    h_out[i]["Y"].copy_(B[i]["Y"], non_blocking=True)
+                    out_y[p][i].record(s_out)
+                for i in reversed(range(nl)):
+                    s_out.wait_event(bwd_done[p][i])
+                    h_out[i]["dX"].copy_(B[i]["dX"], non_blocking=True)
+                    out_dx[p][i].record(s_out)
+                s_out.wait_event(grads_ready)
+                h_grad.copy_(self.bucket, non_blocking=True)
+                grad_out.record(s_out)
+        done_in, done_out = torch.cuda.Event(), torch.cuda.Event()
+        done_in.record(s_in)
+        done_out.record(s_out)
+        main.wait_event(done_in)
+        main.wait_event(done_out)
+        e1.record(main)
+        torch.cuda.synchronize()
+        # the overlapped copies must not have changed the result: the outputs copied out
+        # should equal the device step's (both buffer sets hold the same inputs); the
+        # outcome is reported in the line rather than raised
+        differ = [f"{k}{i}" for i, L in enumerate(self.lin) for k in ("Y", "dX")
+                  if not torch.equal(h_out[i][k], L[k].cpu())]
+        if not torch.equal(h_grad, self.bucket.cpu()):
+            differ.append("grads")
+        self.e2e_differ = differ
+        return e0.elapsed_time(e1), h2d, d2h
+
     def measure(self, steps: int, warmup: int, world: int, local: int, e2e_steps: int = 3) -> dict:
         """Warm-up, K timed steps (barrier + synchronize on both sides, max over
         ranks), a second loop with events around every fused dequant GEMM, and
@@ -455,38 +556,13 @@ class LayerSet:
 
         # end to end through the public API: every linear's X and dY in from pinned
         # host memory, the step, Y, dX and the adapter gradients back out
-        h_in = [{k: torch.empty_like(L[k], device="cpu").pin_memory() for k in ("X", "dY")} for L in self.lin]
-        for h, L in zip(h_in, self.lin):
-            for k in h:
-                h[k].copy_(L[k])
-        h_out = [{k: torch.empty_like(L[k], device="cpu").pin_memory() for k in ("Y", "dX")} for L in self.lin]
-        h_grad = torch.empty_like(self.bucket, device="cpu").pin_memory()
-        h2d = sum(t.numel() * t.element_size() for h in h_in for t in h.values())
-        d2h = sum(t.numel() * t.element_size() for h in h_out for t in h.values()) + h_grad.numel() * 4
-        if world > 1:
-            dist.barrier()
-        torch.cuda.synchronize()
-        e0 = torch.cuda.Event(enable_timing=True)
-        e1 = torch.cuda.Event(enable_timing=True)
-        e0.record()
-        for _ in range(e2e_steps):
-            for h, L in zip(h_in, self.lin):
-                for k in h:
-                    L[k].copy_(h[k], non_blocking=True)
-            one()
-            for h, L in zip(h_out, self.lin):
-                for k in h:
-                    h[k].copy_(L[k], non_blocking=True)
-            h_grad.copy_(self.bucket, non_blocking=True)
-        e1.record()
-        torch.cuda.synchronize()
-        e2e_ms = e0.elapsed_time(e1)
+        e2e_ms, h2d, d2h = self.e2e(e2e_steps, world)
         if world > 1:
             e2e_ms = max_over_ranks(e2e_ms, self.dev)
         self.check("the end-to-end loop")
         return {"ms_step": ms / steps, "fwd_ms": fwd_ms, "bwd_ms": bwd_ms, "launches": int(launches),
                 "clocks": clocks, "e2e_ms_step": e2e_ms / e2e_steps, "e2e_steps": e2e_steps, "h2d": h2d,
-                "d2h": d2h}
+                "d2h": d2h, "e2e_differ": self.e2e_differ}
 
 
 def layer_record(name: str, ls: LayerSet, m: dict, world: int, steps: int, warmup: int) -> dict:
@@ -539,7 +615,10 @@ def layer_record(name: str, ls: LayerSet, m: dict, world: int, steps: int, warmu
                                      f"one capture per weight shape)",
                      "algorithmic_bytes": sum(fused_bytes(c)[0 if dom == "fwd" else 1] for c in ls.cases)},
         "e2e": {"value": round(whole_job_rate(flops, world, m["e2e_ms_step"] * 1e-3) / 1e12, 3), "unit": "TFLOP/s",
-                "h2d_bytes_per_step": m["h2d"], "d2h_bytes_per_step": m["d2h"], "steps": m["e2e_steps"]},
+                "h2d_bytes_per_step": m["h2d"], "d2h_bytes_per_step": m["d2h"], "steps": m["e2e_steps"],
+                "copies": "overlapped with the compute on two copy streams",
+                "outputs_equal_device_step": not m["e2e_differ"],
+                **({"outputs_differing": m["e2e_differ"]} if m["e2e_differ"] else {})},
         "gpu_launches": m["launches"],
         "clocks": m["clocks"],
     }
@@ -561,7 +640,7 @@ def measure_layer_set(name: str, steps: int, warmup: int, world: int, rank: int,
         if not cases:
             raise SystemExit(f"--linear {only}: no such linear in {name}")
     ls = LayerSet(cases, dev, rank, world)
-    m = ls.measure(steps, warmup, world, local)
+    m = ls.measure(steps, warmup, world, local, e2e_steps=max(4, min(10, steps // 2)))
     rec = layer_record(name, ls, m, world, steps, warmup)
     del ls
     torch.cuda.empty_cache()

@@ -74,6 +74,9 @@ struct GemmParams {
   // before the next group, so that the activation tiles the resident CTAs share
   // stay in L2 while the W tiles stream past them.
   int raster_gm;
+  // gemm_kernel only: 1 = let the next grid start early (programmatic launch);
+  // set only where the small-M forward follows.
+  int trigger_dependents;
 };
 
 template <int BN_, int STAGES_, bool A_MN_, int BMODE_, int LORA_, int OUT_>
@@ -159,7 +162,16 @@ __global__ void __launch_bounds__(C::NUM_THREADS, 1)
   const uint32_t tmem_acc = *tmem_slot;
   const uint32_t smem_base = smem_u32(smem);
   pdl_wait();  // inputs of this grid were written by earlier grids of the stream
-  pdl_launch_dependents();
+  // Early trigger only where the small-M forward follows.  Elsewhere the next grid
+  // (above all the CTA-pair GEMM after s·X·A or s·dY·Bᵀ) becomes resident only when
+  // this one has finished: with the trigger, the CTA-pair GEMM produced run-to-run
+  // different outputs (one output column of a 512-token tile, in a few launches per
+  // hundred) although every one of its CTAs waits for this grid before touching
+  // memory; without it, and with programmatic launch switched off altogether,
+  // thousands of repeated calls were bit-identical.  The small-M kernel after an
+  // early trigger was bit-identical in the same test and gains the overlap (its
+  // forward is 27 instead of 36 µs for 8192 x 8192 at 16 tokens).
+  if (p.trigger_dependents) pdl_launch_dependents();
 
   if (warp == 0) {
     // ------------------------------------------------------------ TMA producer

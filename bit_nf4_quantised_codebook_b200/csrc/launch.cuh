@@ -1,13 +1,15 @@
 // launch.cuh — every kernel of the library is launched through launch_k():
 // cudaLaunchKernelEx with programmatic dependent launch enabled (and, for the
 // skinny GEMMs, a 1 x 1 x cz cluster).  Each kernel calls pdl_wait() before its
-// first access to global memory and pdl_launch_dependents() right after it, so
-// the next kernel's CTAs can be placed and run their prologue (barrier init,
-// TMEM allocation, tensor-map prefetch) while this one runs; stream order for
-// memory is unchanged.  Because a kernel triggers its dependents only after its
-// own wait returned, every grid before its predecessor is complete when a
-// dependent starts: a dependent that reads some inputs before its own wait may
-// rely on that (it must still wait before reading its predecessor's output).
+// first access to global memory, and most call pdl_launch_dependents() right
+// after it, so the next kernel's CTAs can be placed and run their prologue
+// (barrier init, TMEM allocation, tensor-map prefetch) while this one runs;
+// stream order for memory is unchanged.  The kernels of gemm.cuh do not trigger
+// early (see there): the grid after them starts when they have finished.
+// Because a kernel triggers its dependents only after its own wait returned,
+// every grid before its predecessor is complete when a dependent starts: a
+// dependent that reads some inputs before its own wait may rely on that (it must
+// still wait before reading its predecessor's output).
 #pragma once
 #include <atomic>
 #include <cstdint>

@@ -143,8 +143,9 @@ static GemmParams base_params(const LaunchCtx &c) {
 // reduction split over the sp.splits CTAs of one cluster and summed in-cluster.
 // Writes out[row][c] (ld_out) or, for SK_DB, out[c][row].
 static cudaError_t run_skinny(SkinnyKind kind, const LaunchCtx &c, const SplitPlan &sp, int rpad, int r, int rows,
-                              float scale, const TmaMaps &maps, void *out, int64_t ld_out) {
+                              float scale, const TmaMaps &maps, void *out, int64_t ld_out, bool trigger = false) {
   GemmParams p = base_params(c);
+  p.trigger_dependents = trigger ? 1 : 0;
   p.rows = rows;
   p.cols = rpad;
   p.k_iters = sp.k_iters;
@@ -300,12 +301,12 @@ static cudaError_t run_small_forward(const LaunchCtx &c, const qlora_nf4_weight 
 // ---------------------------------------------------------------- forward
 // sT = bf16(s·X·A)  (A-op X [M,K] K-major; B-op Aᵀ: A [K,r] read MN-major)
 static cudaError_t run_t(const LaunchCtx &c, const uint16_t *X, int64_t M, int K, const uint16_t *A, int r, float s,
-                         uint16_t *sT, const LinearPlan &pl) {
+                         uint16_t *sT, const LinearPlan &pl, bool trigger) {
   TmaMaps m;
   if (!map_bf16_kmajor(&m.a, X, K, M, 128) || !map_bf16_mn(&m.b, A, r, K)) return cudaErrorInvalidValue;
   m.a2 = m.a;
   m.b2 = m.b;
-  return run_skinny(SK_T, c, pl.sp_t, pl.rpad, r, static_cast<int>(M), s, m, sT, r);
+  return run_skinny(SK_T, c, pl.sp_t, pl.rpad, r, static_cast<int>(M), s, m, sT, r, trigger);
 }
 
 cudaError_t run_forward(const LaunchCtx &c, const qlora_nf4_weight &w, const uint16_t *X, int64_t M,
@@ -314,7 +315,8 @@ cudaError_t run_forward(const LaunchCtx &c, const qlora_nf4_weight &w, const uin
   cudaError_t e;
   const int K = static_cast<int>(w.K);
   uint16_t *sT = T_save ? T_save : reinterpret_cast<uint16_t *>(ws + pl.off_sT);
-  if ((e = run_t(c, X, M, K, A, r, s, sT, pl)) != cudaSuccess) return e;
+  // the small-M forward that follows overlaps this grid's tail; the CTA-pair GEMM does not (gemm.cuh)
+  if ((e = run_t(c, X, M, K, A, r, s, sT, pl, pl.small_main)) != cudaSuccess) return e;
   // Y = X·W_hatᵀ + sT·B
   const TimingHooks &hk = timing_hooks();
   if (pl.small_main) return run_small_forward(c, w, X, M, sT, B, r, Y, pl.sp_main, hk.fwd_begin, hk.fwd_end);
@@ -331,7 +333,7 @@ cudaError_t run_backward(const LaunchCtx &c, const qlora_nf4_weight &w, const ui
   const uint16_t *sT = T_saved;
   if (!sT) {  // recompute bf16(s·X·A)
     uint16_t *sT_ws = reinterpret_cast<uint16_t *>(ws + pl.off_sT);
-    if ((e = run_t(c, X, M, K, A, r, s, sT_ws, pl)) != cudaSuccess) return e;
+    if ((e = run_t(c, X, M, K, A, r, s, sT_ws, pl, false)) != cudaSuccess) return e;
     sT = sT_ws;
   }
   uint16_t *sU = reinterpret_cast<uint16_t *>(ws + pl.off_sU);
