@@ -82,17 +82,19 @@ def _peaks():
 # set (q, gate and down: k, v and o share q's shape, up shares gate's).  A set's
 # figure is the sum over its linears.
 KERNEL_SOURCES = ["gemm_pair.cuh", "gemm.cuh", "nf4_decode.cuh", "ptx.cuh", "launch.cuh", "linear.cu"]
-TRAFFIC_CAPTURE = {"sources_sha1": "d1e611bffc63fb7fa183aa54d0ae0d3bc560c901",
-                   ("shapes_65b", 8192, 8192, "fwd"): 526_467_840, ("shapes_65b", 8192, 8192, "bwd"): 497_913_856,
-                   ("shapes_65b", 22016, 8192, "fwd"): 1_031_215_872,
-                   ("shapes_65b", 22016, 8192, "bwd"): 1_419_983_360,
-                   ("shapes_65b", 8192, 22016, "fwd"): 1_412_864_512,
-                   ("shapes_65b", 8192, 22016, "bwd"): 1_060_189_696,
-                   ("llama7b_layer", 4096, 4096, "fwd"): 46_133_248, ("llama7b_layer", 4096, 4096, "bwd"): 44_052_736,
-                   ("llama7b_layer", 11008, 4096, "fwd"): 118_332_928,
-                   ("llama7b_layer", 11008, 4096, "bwd"): 194_748_928,
-                   ("llama7b_layer", 4096, 11008, "fwd"): 198_091_008,
-                   ("llama7b_layer", 4096, 11008, "bwd"): 114_373_888}
+TRAFFIC_CAPTURE = {"sources_sha1": "f0d2ab5405988ee0360c99b2b8ffa1cfa4835f1e",
+                   ("shapes_65b", 8192, 8192, "fwd"): 539_570_944,
+                   ("shapes_65b", 8192, 8192, "bwd"): 535_533_824,
+                   ("shapes_65b", 22016, 8192, "fwd"): 1_105_506_048,
+                   ("shapes_65b", 22016, 8192, "bwd"): 1_421_735_680,
+                   ("shapes_65b", 8192, 22016, "fwd"): 1_415_080_704,
+                   ("shapes_65b", 8192, 22016, "bwd"): 1_208_976_128,
+                   ("llama7b_layer", 4096, 4096, "fwd"): 46_345_472,
+                   ("llama7b_layer", 4096, 4096, "bwd"): 44_085_248,
+                   ("llama7b_layer", 11008, 4096, "fwd"): 118_707_968,
+                   ("llama7b_layer", 11008, 4096, "bwd"): 197_318_912,
+                   ("llama7b_layer", 4096, 11008, "fwd"): 196_402_176,
+                   ("llama7b_layer", 4096, 11008, "bwd"): 117_616_896}
 # The small-M kernel: the same one-pass capture of `--workload smallm`, bytes per launch, per (N, M).
 SMALLM_SOURCES = ["gemm_smallm.cuh", "gemm.cuh", "nf4_decode.cuh", "ptx.cuh", "launch.cuh", "linear.cu"]
 SMALLM_TRAFFIC = {"sources_sha1": None}

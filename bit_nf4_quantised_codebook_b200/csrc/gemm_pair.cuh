@@ -148,7 +148,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(C::NUM_THREADS, 1)
   const uint32_t tmem_acc = *tmem_slot;
   const uint32_t smem_base = smem_u32(smem);
   pdl_wait();  // inputs of this grid were written by earlier grids of the stream
-  pdl_launch_dependents();
+  // No early trigger either: the grid after this one starts when it has finished
+  // (see gemm.cuh on run-to-run differences seen with early triggers around this kernel).
 
   if (warp == 0) {
     // ------------------------------------------------------------ A producer

@@ -4,8 +4,9 @@
 // first access to global memory, and most call pdl_launch_dependents() right
 // after it, so the next kernel's CTAs can be placed and run their prologue
 // (barrier init, TMEM allocation, tensor-map prefetch) while this one runs;
-// stream order for memory is unchanged.  The kernels of gemm.cuh do not trigger
-// early (see there): the grid after them starts when they have finished.
+// stream order for memory is unchanged.  The kernels of gemm.cuh and
+// gemm_pair.cuh do not trigger early (see gemm.cuh): the grid after them starts
+// when they have finished, except that s·X·A lets the small-M forward start early.
 // Because a kernel triggers its dependents only after its own wait returned,
 // every grid before its predecessor is complete when a dependent starts: a
 // dependent that reads some inputs before its own wait may rely on that (it must
