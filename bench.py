@@ -80,7 +80,10 @@ def _peaks():
 # --no-cpu-baseline --steps 3 --warmup 3` (one linear per step; the capture is the
 # first timed step's forward and backward launch), one run per weight shape of the
 # set (q, gate and down: k, v and o share q's shape, up shares gate's).  A set's
-# figure is the sum over its linears.
+# figure is the sum over its linears.  The 7B projection's two entries come from
+# the launch list of `bench.py --workload proj7b --no-sub --no-cpu-baseline
+# --steps 2 --warmup 3` (the same metrics, `-s 21 -c 6`: one step after the load
+# and warm-up launches).
 KERNEL_SOURCES = ["gemm_pair.cuh", "gemm.cuh", "nf4_decode.cuh", "ptx.cuh", "launch.cuh", "linear.cu"]
 TRAFFIC_CAPTURE = {"sources_sha1": "f0d2ab5405988ee0360c99b2b8ffa1cfa4835f1e",
                    ("shapes_65b", 8192, 8192, "fwd"): 539_570_944,
@@ -94,7 +97,9 @@ TRAFFIC_CAPTURE = {"sources_sha1": "f0d2ab5405988ee0360c99b2b8ffa1cfa4835f1e",
                    ("llama7b_layer", 11008, 4096, "fwd"): 118_707_968,
                    ("llama7b_layer", 11008, 4096, "bwd"): 197_318_912,
                    ("llama7b_layer", 4096, 11008, "fwd"): 196_402_176,
-                   ("llama7b_layer", 4096, 11008, "bwd"): 117_616_896}
+                   ("llama7b_layer", 4096, 11008, "bwd"): 117_616_896,
+                   ("proj7b", 4096, 4096, "fwd"): 44_851_200,
+                   ("proj7b", 4096, 4096, "bwd"): 45_932_288}
 # The small-M kernel: the same one-pass capture of `--workload smallm`, bytes per launch, per (N, M).
 SMALLM_SOURCES = ["gemm_smallm.cuh", "gemm.cuh", "nf4_decode.cuh", "ptx.cuh", "launch.cuh", "linear.cu"]
 SMALLM_TRAFFIC = {"sources_sha1": None}
