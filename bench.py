@@ -100,13 +100,18 @@ TRAFFIC_CAPTURE = {"sources_sha1": "f0d2ab5405988ee0360c99b2b8ffa1cfa4835f1e",
                    ("llama7b_layer", 4096, 11008, "bwd"): 117_616_896,
                    ("proj7b", 4096, 4096, "fwd"): 44_851_200,
                    ("proj7b", 4096, 4096, "bwd"): 45_932_288}
-# The small-M kernel: the same one-pass capture of `--workload smallm`, bytes per launch, per (N, M).
+# The small-M kernel, bytes per launch, per (N, M): the same three metrics with
+# `-k regex:smallm -s 3 -c 1` over `bench.py --workload smallm --n N --m M --steps 5
+# --warmup 3 --no-cpu-baseline`.
 SMALLM_SOURCES = ["gemm_smallm.cuh", "gemm.cuh", "nf4_decode.cuh", "ptx.cuh", "launch.cuh", "linear.cu"]
-SMALLM_TRAFFIC = {"sources_sha1": None}
-# The AdamW kernel: the same capture of `--workload adamw`, bytes per launch (the 150 MB working
-# set is only a little larger than L2, so part of the writes stay in L2).
+SMALLM_TRAFFIC = {"sources_sha1": "c299ca6592e319c5c83b38ed8b1ad3e1d83af7dd",
+                  (8192, 1): 35_737_856, (8192, 16): 35_979_264,
+                  (28672, 1): 128_225_536, (28672, 16): 128_480_768}
+# The AdamW kernel, bytes per launch: `-k regex:adamw -s 3 -c 1` over `bench.py --workload adamw
+# --steps 3 --warmup 3 --no-cpu-baseline` (the 150 MB working set is only a little larger than
+# L2, so part of the writes stay in L2).
 ADAMW_SOURCES = ["adamw.cu", "ptx.cuh", "launch.cuh"]
-ADAMW_TRAFFIC = {"sources_sha1": "0064428f763192ff27c64743df1b67afd4a73e71", "bytes": 90_732_000}
+ADAMW_TRAFFIC = {"sources_sha1": "587ae2e8636866758a5884b157e140ce9bc47283", "bytes": 97_109_760}
 
 
 def kernel_sources_sha1(files=None) -> str:
@@ -1117,10 +1122,11 @@ def run_adamw(args):
 
 MERGE_SHAPES = ADAMW_SHAPES  # the seven linears of one LLaMA-7B decoder layer
 # ncu DRAM read + write of the merge-and-code kernel over one step's seven launches (a one-pass
-# `--metrics gpu__time_duration.sum,dram__bytes_read.sum,dram__bytes_write.sum -k regex:merge`
-# capture of `--workload merge`), valid for the sources it was taken from.
+# `--metrics gpu__time_duration.sum,dram__bytes_read.sum,dram__bytes_write.sum -k regex:merge
+# -s 21 -c 7` capture of `bench.py --workload merge --steps 3 --warmup 3 --no-cpu-baseline`),
+# valid for the sources it was taken from.
 MERGE_SOURCES = ["merge.cu", "nf4_decode.cuh", "nf4_quant.cuh", "ptx.cuh", "launch.cuh"]
-MERGE_TRAFFIC = {"sources_sha1": "4e714f616c7e4e56f4c0d477b522210425681dd2", "bytes_per_step": 117_096_000}
+MERGE_TRAFFIC = {"sources_sha1": "baec0f2d4c3e0bb75eea6544f7cf2063a5f6b3f3", "bytes_per_step": 117_138_432}
 
 
 def merge_bytes(N: int, K: int, r: int) -> int:
