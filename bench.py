@@ -683,9 +683,9 @@ def measure_smallm(n: int, m_tok: int, steps: int, warmup: int, world: int, loca
                      device=dev)
     err = api.new_error_word(dev)
 
-    def step(i, Xin=None):
-        api.qlora_linear_forward(qs[i % ncopy], X if Xin is None else Xin, A, B, s, Y=Y, T_save=sT, ws=ws,
-                                 dev_err=err)
+    def step(i, Xin=None, Yout=None):
+        api.qlora_linear_forward(qs[i % ncopy], X if Xin is None else Xin, A, B, s, Y=Y if Yout is None else Yout,
+                                 T_save=sT, ws=ws, dev_err=err)
 
     for i in range(warmup):
         step(i)
@@ -725,22 +725,48 @@ def measure_smallm(n: int, m_tok: int, steps: int, warmup: int, world: int, loca
         raise RuntimeError(f"device error word {int(err[0].item())}")
     ms_step = ms / steps
 
-    # end to end: X host -> device, forward, Y device -> host
+    # end to end: X host -> device, forward, Y device -> host, every step.  The copies
+    # run on one stream of their own, so they overlap the forwards around them; X and
+    # Y are double buffered by step parity.  Per step i the copy stream waits for
+    # forward i, copies Y_i out and X_{i+2} in (into forward i's X buffer), so forward
+    # i+2 (which waits for that X) also finds Y_i's buffer copied out.  Two event
+    # records and two waits per step keep the host's share of a step small.
     e2e_steps = e2e_steps or max(3, min(100, steps // 10))
     hx = X.cpu().pin_memory()
     hy = torch.empty_like(Y, device="cpu").pin_memory()
-    dx = torch.empty_like(X)
+    dxs = [torch.empty_like(X) for _ in range(2)]
+    dys = [torch.empty_like(Y) for _ in range(2)]
+    main = torch.cuda.current_stream()
+    s_copy = torch.cuda.Stream()
+    x_in = [torch.cuda.Event() for _ in range(e2e_steps)]  # X of step i landed
+    fwd = [torch.cuda.Event() for _ in range(e2e_steps)]   # forward of step i done
     torch.cuda.synchronize()
     e0 = torch.cuda.Event(enable_timing=True)
     e1 = torch.cuda.Event(enable_timing=True)
-    e0.record()
+    e0.record(main)
+    s_copy.wait_event(e0)
+    with torch.cuda.stream(s_copy):
+        for i in range(min(2, e2e_steps)):
+            dxs[i].copy_(hx, non_blocking=True)
+            x_in[i].record(s_copy)
     for i in range(e2e_steps):
-        dx.copy_(hx, non_blocking=True)
-        step(i, dx)
-        hy.copy_(Y, non_blocking=True)
-    e1.record()
+        p = i % 2
+        main.wait_event(x_in[i])
+        step(i, dxs[p], dys[p])
+        fwd[i].record(main)
+        s_copy.wait_event(fwd[i])
+        with torch.cuda.stream(s_copy):
+            hy.copy_(dys[p], non_blocking=True)
+            if i + 2 < e2e_steps:
+                dxs[p].copy_(hx, non_blocking=True)
+                x_in[i + 2].record(s_copy)
+    done = torch.cuda.Event()
+    done.record(s_copy)
+    main.wait_event(done)
+    e1.record(main)
     torch.cuda.synchronize()
     e2e_ms = e0.elapsed_time(e1) / e2e_steps
+    e2e_equal = torch.equal(hy, Y.cpu())  # the copied-out Y equals the device loop's
     del qs
     torch.cuda.empty_cache()
 
@@ -763,7 +789,8 @@ def measure_smallm(n: int, m_tok: int, steps: int, warmup: int, world: int, loca
                      "traffic": _traffic(SMALLM_TRAFFIC, SMALLM_SOURCES, (N, M)),
                      "traffic_unit": "bytes per launch (ncu dram read+write)"},
         "e2e": {"value": round(packed / (e2e_ms * 1e-3) / 1e9, 2), "unit": "GB/s",
-                "h2d_bytes_per_step": X.numel() * 2, "d2h_bytes_per_step": Y.numel() * 2, "steps": e2e_steps},
+                "h2d_bytes_per_step": X.numel() * 2, "d2h_bytes_per_step": Y.numel() * 2, "steps": e2e_steps,
+                "copies": "overlapped with the compute on two copy streams", "outputs_equal_device_step": e2e_equal},
         "gpu_launches": int(launches),
         "clocks": clocks,
     }
@@ -823,26 +850,51 @@ def run_quantiser(args):
     clocks = sampler.stop()
     by = 2 * n * k + api.alloc_weight(n, k).nbytes()
     dev = torch.device("cuda", local)
-    # end to end: the bf16 weight host -> device, quantise, the stored weight device -> host
-    W = api.bits_to_tensor(inputs.weight_bf16(n, k, 0.015, 0, 0.001), dev)
-    hw = W.cpu().pin_memory()
-    wq = api.alloc_weight(n, k, dev)
+    # end to end: the bf16 weight host -> device, quantise, the stored weight device ->
+    # host, every call; the copies on two streams of their own, overlapping the calls
+    # around them, with the device weight and its stored form double buffered
+    hw = api.bits_to_tensor(inputs.weight_bf16(n, k, 0.015, 0, 0.001), dev).cpu().pin_memory()
+    Ws = [torch.empty_like(hw, device=dev) for _ in range(2)]
+    wqs = [api.alloc_weight(n, k, dev) for _ in range(2)]
     ws = torch.empty(api.qlora_workspace_size(api.QLORA_OP_QUANTIZE, 0, n, k, 0), dtype=torch.uint8, device=dev)
-    outs = [torch.empty_like(t, device="cpu").pin_memory() for t in (wq.codes, wq.c2q, wq.c1, wq.mean)]
+    outs = [torch.empty_like(t, device="cpu").pin_memory() for t in (wqs[0].codes, wqs[0].c2q, wqs[0].c1, wqs[0].mean)]
     e2e_steps = 5
+    main = torch.cuda.current_stream()
+    s_in, s_out = torch.cuda.Stream(), torch.cuda.Stream()
+    w_in, q_done, q_out = ([torch.cuda.Event() for _ in range(2)] for _ in range(3))
     torch.cuda.synchronize()
     e0 = torch.cuda.Event(enable_timing=True)
     e1 = torch.cuda.Event(enable_timing=True)
     launches0 = api.qlora_kernel_launch_count()
-    e0.record()
-    for _ in range(e2e_steps):
-        W.copy_(hw, non_blocking=True)
-        api.qlora_quantize(W, out=wq, ws=ws)
-        for h, d in zip(outs, (wq.codes, wq.c2q, wq.c1, wq.mean)):
-            h.copy_(d, non_blocking=True)
-    e1.record()
+    e0.record(main)
+    s_in.wait_event(e0)
+    s_out.wait_event(e0)
+    for i in range(e2e_steps):
+        p = i % 2
+        with torch.cuda.stream(s_in):
+            if i >= 2:
+                s_in.wait_event(q_done[p])  # the call two back has read this weight buffer
+            Ws[p].copy_(hw, non_blocking=True)
+            w_in[p].record(s_in)
+        main.wait_event(w_in[p])
+        if i >= 2:
+            main.wait_event(q_out[p])  # the stored weight of two calls back has been copied out
+        api.qlora_quantize(Ws[p], out=wqs[p], ws=ws)
+        q_done[p].record(main)
+        with torch.cuda.stream(s_out):
+            s_out.wait_event(q_done[p])
+            for h, d in zip(outs, (wqs[p].codes, wqs[p].c2q, wqs[p].c1, wqs[p].mean)):
+                h.copy_(d, non_blocking=True)
+            q_out[p].record(s_out)
+    done = torch.cuda.Event()
+    done.record(s_out)
+    main.wait_event(done)
+    e1.record(main)
     torch.cuda.synchronize()
     e2e_ms = e0.elapsed_time(e1) / e2e_steps
+    wq = wqs[(e2e_steps - 1) % 2]
+    other = wqs[e2e_steps % 2]  # the same weight quantised by another call (two calls back)
+    e2e_equal = all(torch.equal(h, d.cpu()) for h, d in zip(outs, (other.codes, other.c2q, other.c1, other.mean)))
     launches = (api.qlora_kernel_launch_count() - launches0) // e2e_steps * args.steps
     hbm, _, _, peak_src = _peaks()
     line = {
@@ -859,7 +911,8 @@ def run_quantiser(args):
                      "unit": "GB/s", "frac": q["hbm_frac"], "peak_source": f"{peak_src} HBM copy", "traffic": None,
                      "traffic_unit": "bytes per call (ncu dram read+write)"},
         "e2e": {"value": round(by / (e2e_ms * 1e-3) / 1e9, 2), "unit": "GB/s", "h2d_bytes_per_step": 2 * n * k,
-                "d2h_bytes_per_step": wq.nbytes(), "steps": e2e_steps},
+                "d2h_bytes_per_step": wq.nbytes(), "steps": e2e_steps,
+                "copies": "overlapped with the compute on two copy streams", "outputs_equal_device_step": e2e_equal},
         "gpu_launches": int(launches),
         "clocks": clocks,
     }
