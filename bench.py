@@ -790,7 +790,7 @@ def measure_smallm(n: int, m_tok: int, steps: int, warmup: int, world: int, loca
                      "traffic_unit": "bytes per launch (ncu dram read+write)"},
         "e2e": {"value": round(packed / (e2e_ms * 1e-3) / 1e9, 2), "unit": "GB/s",
                 "h2d_bytes_per_step": X.numel() * 2, "d2h_bytes_per_step": Y.numel() * 2, "steps": e2e_steps,
-                "copies": "overlapped with the compute on two copy streams", "outputs_equal_device_step": e2e_equal},
+                "copies": "overlapped with the compute on one copy stream", "outputs_equal_device_step": e2e_equal},
         "gpu_launches": int(launches),
         "clocks": clocks,
     }
