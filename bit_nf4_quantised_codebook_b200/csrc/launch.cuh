@@ -7,6 +7,8 @@
 // stream order for memory is unchanged.  The kernels of gemm.cuh and
 // gemm_pair.cuh do not trigger early (see gemm.cuh): the grid after them starts
 // when they have finished, except that s·X·A lets the small-M forward start early.
+// They are also launched without the programmatic attribute (launch_k_ordered),
+// the small-M forward with it.
 // Because a kernel triggers its dependents only after its own wait returned,
 // every grid before its predecessor is complete when a dependent starts: a
 // dependent that reads some inputs before its own wait may rely on that (it must
@@ -36,8 +38,8 @@ inline cudaError_t smem_attr_once(const void *kern, int bytes, std::atomic<uint6
 }
 
 template <typename... KArgs, typename... Args>
-cudaError_t launch_k(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st, unsigned cz,
-                     Args &&...args) {
+cudaError_t launch_k_pdl(bool pdl, void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st,
+                         unsigned cz, Args &&...args) {
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = grid;
   cfg.blockDim = block;
@@ -46,7 +48,7 @@ cudaError_t launch_k(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem,
   cudaLaunchAttribute attr[2];
   unsigned n = 0;
   attr[n].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-  attr[n].val.programmaticStreamSerializationAllowed = 1;
+  attr[n].val.programmaticStreamSerializationAllowed = pdl ? 1 : 0;
   ++n;
   if (cz > 1) {
     attr[n].id = cudaLaunchAttributeClusterDimension;
@@ -63,6 +65,22 @@ cudaError_t launch_k(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem,
   // reported again by the next one
   const cudaError_t last = cudaGetLastError();
   return e != cudaSuccess ? e : last;
+}
+
+// Programmatic dependent launch on: the kernel may start as soon as its predecessor
+// triggers (it still waits for it before touching memory).
+template <typename... KArgs, typename... Args>
+cudaError_t launch_k(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st, unsigned cz,
+                     Args &&...args) {
+  return launch_k_pdl(true, kern, grid, block, smem, st, cz, std::forward<Args>(args)...);
+}
+
+// Plain stream order: the kernel starts when its predecessor has finished.  Used for
+// the dequant and adapter GEMMs (gemm.cuh, gemm_pair.cuh).
+template <typename... KArgs, typename... Args>
+cudaError_t launch_k_ordered(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st,
+                             unsigned cz, Args &&...args) {
+  return launch_k_pdl(false, kern, grid, block, smem, st, cz, std::forward<Args>(args)...);
 }
 
 }  // namespace qlora

@@ -52,7 +52,8 @@ template <class C>
 static cudaError_t launch(dim3 grid, const TmaMaps &m, const GemmParams &p, cudaStream_t st) {
   cudaError_t e = prepare<C>();
   if (e != cudaSuccess) return e;
-  return launch_k(gemm_kernel<C>, grid, dim3(C::NUM_THREADS), C::SMEM_BYTES, st, 1, m.a, m.b, m.a2, m.b2, p);
+  return launch_k_ordered(gemm_kernel<C>, grid, dim3(C::NUM_THREADS), C::SMEM_BYTES, st, 1, m.a, m.b, m.a2, m.b2,
+                          p);
 }
 
 // Launch with clusters of 1 x 1 x cz CTAs (the K splits of one output tile).
@@ -60,7 +61,7 @@ template <class C>
 static cudaError_t launch_cluster(dim3 grid, int cz, const TmaMaps &m, const GemmParams &p, cudaStream_t st) {
   cudaError_t e = prepare<C>();
   if (e != cudaSuccess) return e;
-  return launch_k(gemm_kernel<C>, grid, dim3(C::NUM_THREADS), C::SMEM_BYTES, st, static_cast<unsigned>(cz), m.a,
+  return launch_k_ordered(gemm_kernel<C>, grid, dim3(C::NUM_THREADS), C::SMEM_BYTES, st, static_cast<unsigned>(cz), m.a,
                   m.b, m.a2, m.b2, p);
 }
 
@@ -75,7 +76,8 @@ static cudaError_t launch_pair(dim3 grid, const TmaMaps &m, const GemmParams &p,
   static std::atomic<uint64_t> prepared{0};
   cudaError_t e = smem_attr_once(reinterpret_cast<const void *>(gemm_pair_kernel<C>), C::SMEM_BYTES, prepared);
   if (e != cudaSuccess) return e;
-  return launch_k(gemm_pair_kernel<C>, grid, dim3(C::NUM_THREADS), C::SMEM_BYTES, st, 1, m.a, m.b, m.a2, m.b2, p);
+  return launch_k_ordered(gemm_pair_kernel<C>, grid, dim3(C::NUM_THREADS), C::SMEM_BYTES, st, 1, m.a, m.b, m.a2,
+                          m.b2, p);
 }
 
 // ---------------------------------------------------------------- finalize kernels
