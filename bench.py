@@ -74,6 +74,9 @@ def _peaks():
 # DRAM traffic (ncu dram__bytes_read.sum + dram__bytes_write.sum) of the dominant
 # kernels, from one-pass ncu launch-list captures, reported only while the kernel
 # sources hash to the build each capture was taken of (otherwise null).
+# Source hashes below were renewed once without a new capture, after the GEMMs'
+# launches switched to plain stream order: a host-side launch attribute, with the
+# kernels, their grids and tiles unchanged, so the bytes per launch are too.
 # Fused dequant GEMMs, bytes per launch, keyed by (layer set, N, K, "fwd" | "bwd"):
 # `ncu --metrics gpu__time_duration.sum,dram__bytes_read.sum,dram__bytes_write.sum
 # --clock-control none -k regex:gemm_pair -s 6 -c 2` over `bench.py --linear <name>
@@ -85,7 +88,7 @@ def _peaks():
 # --steps 2 --warmup 3` (the same metrics, `-s 21 -c 6`: one step after the load
 # and warm-up launches).
 KERNEL_SOURCES = ["gemm_pair.cuh", "gemm.cuh", "nf4_decode.cuh", "ptx.cuh", "launch.cuh", "linear.cu"]
-TRAFFIC_CAPTURE = {"sources_sha1": "f0d2ab5405988ee0360c99b2b8ffa1cfa4835f1e",
+TRAFFIC_CAPTURE = {"sources_sha1": "b40d0bee28beb57f87da184c3853be6494423554",
                    ("shapes_65b", 8192, 8192, "fwd"): 539_570_944,
                    ("shapes_65b", 8192, 8192, "bwd"): 535_533_824,
                    ("shapes_65b", 22016, 8192, "fwd"): 1_105_506_048,
@@ -104,14 +107,14 @@ TRAFFIC_CAPTURE = {"sources_sha1": "f0d2ab5405988ee0360c99b2b8ffa1cfa4835f1e",
 # `-k regex:smallm -s 3 -c 1` over `bench.py --workload smallm --n N --m M --steps 5
 # --warmup 3 --no-cpu-baseline`.
 SMALLM_SOURCES = ["gemm_smallm.cuh", "gemm.cuh", "nf4_decode.cuh", "ptx.cuh", "launch.cuh", "linear.cu"]
-SMALLM_TRAFFIC = {"sources_sha1": "c299ca6592e319c5c83b38ed8b1ad3e1d83af7dd",
+SMALLM_TRAFFIC = {"sources_sha1": "a8228d129df7c1a36e47db167baba47c3046508d",
                   (8192, 1): 35_737_856, (8192, 16): 35_979_264,
                   (28672, 1): 128_225_536, (28672, 16): 128_480_768}
 # The AdamW kernel, bytes per launch: `-k regex:adamw -s 3 -c 1` over `bench.py --workload adamw
 # --steps 3 --warmup 3 --no-cpu-baseline` (the 150 MB working set is only a little larger than
 # L2, so part of the writes stay in L2).
 ADAMW_SOURCES = ["adamw.cu", "ptx.cuh", "launch.cuh"]
-ADAMW_TRAFFIC = {"sources_sha1": "587ae2e8636866758a5884b157e140ce9bc47283", "bytes": 97_109_760}
+ADAMW_TRAFFIC = {"sources_sha1": "4fff1a2cc2a9bff24c7253a43f3cd653498792f8", "bytes": 97_109_760}
 
 
 def kernel_sources_sha1(files=None) -> str:
@@ -1179,7 +1182,7 @@ MERGE_SHAPES = ADAMW_SHAPES  # the seven linears of one LLaMA-7B decoder layer
 # -s 21 -c 7` capture of `bench.py --workload merge --steps 3 --warmup 3 --no-cpu-baseline`),
 # valid for the sources it was taken from.
 MERGE_SOURCES = ["merge.cu", "nf4_decode.cuh", "nf4_quant.cuh", "ptx.cuh", "launch.cuh"]
-MERGE_TRAFFIC = {"sources_sha1": "baec0f2d4c3e0bb75eea6544f7cf2063a5f6b3f3", "bytes_per_step": 117_138_432}
+MERGE_TRAFFIC = {"sources_sha1": "e700d8e13803ffca02afa8d12ef8424109bd85c8", "bytes_per_step": 117_138_432}
 
 
 def merge_bytes(N: int, K: int, r: int) -> int:
