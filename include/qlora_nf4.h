@@ -219,7 +219,7 @@ qlora_status qlora_linear_forward(const qlora_nf4_weight *w, const uint16_t *X, 
                                   int *dev_err, void *stream);
 
 /*
- * qlora_linear_backward — §The QLoRA layer, end to end (backward listing).
+ * qlora_linear_backward — §The QLoRA layer, end to end (backward).
  *   U  = dY·Bᵀ                                   (M x r)
  *   dX = dY·W_hat + bf16(s·U)·Aᵀ                 (M x K bfloat16; nullable = skip)
  *   dA = Xᵀ·bf16(s·U)                            (K x r float32)
